@@ -1,0 +1,491 @@
+"""Benchmark of the weight-only NVFP4 GEMV decode-step sweep on B200.
+
+One step = the decode-step sweep: 4 synthetic layers, each with qkv (10240x5120), o (5120x6144),
+the fused gate_up dual (2 x 17408x5120) and down (5120x17408) NVFP4 projections, run back to back
+on one stream, for every row count M in {1, 2, 4, 8} -- 64 launches, 3.16 GB of packed weights
+and scales streamed per step (0.79 GB per M pass, far above the 126 MB L2, so no flush is needed).
+
+Metric: effective HBM GB/s = (packed weights + scales + bf16 activations + bf16 outputs) bytes
+per step / device time per step.  Printed as one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs an independent replica on its own GPU (the GEMV needs no
+collective); value = bytes of all ranks / max over ranks of the device time.
+--impl reference times the CPU fp64 oracle (the plain C reference) on a bounded sample of the
+same workload on rank 0's host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "sweep"
+METRIC = "NVFP4 GEMV effective HBM GB/s and % of B200 peak, rows 1/8"
+WORKLOAD_DESC = ("decode-step sweep: 4 layers x {qkv 10240x5120, o 5120x6144, gate_up dual "
+                 "2x17408x5120, down 5120x17408} NVFP4, M in {1,2,4,8}, back to back on one stream")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-steps", type=int, default=0,
+                    help="run this many eager steps and exit (for ncu launch lists)")
+    return ap.parse_args()
+
+
+def step_bytes(wl) -> dict:
+    """Algorithmic bytes per launch, keyed by (projection, M)."""
+    out = {}
+    for m in wl.rows:
+        for p in wl.projections:
+            nw = 2 if p.dual else 1
+            out[(p.name, m)] = nw * (p.n * p.k // 2 + p.n * p.k // 16) + m * p.k * 2 + m * p.n * 2
+    return out
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------------------------
+# clocks
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            f = [t.strip() for t in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        # samples under load: the top half by clock is not a filter we want; keep them all
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+
+
+def dist_setup(gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world <= 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+
+
+def cpu_oracle_sample(wl, seconds: float):
+    """Time the fp64 oracle on row slices of the workload's projections (rank 0, host cores)."""
+    import oracle
+    oracle.build()
+    threads = os.cpu_count() or 1
+    done_bytes, t_total, calls = 0, 0.0, []
+    rng = np.random.default_rng(0)
+    order = [(p, m) for m in wl.rows for p in wl.projections]
+    i = 0
+    while t_total < seconds and i < 4 * len(order):
+        p, m = order[i % len(order)]
+        i += 1
+        rows = np.arange(0, min(p.n, 256)) + int(rng.integers(0, max(1, p.n - 256)))
+        t0 = time.perf_counter()
+        if p.dual:
+            oracle.gemv_dual(p.w.packed, p.w.scales, p.w.g, p.w_up.packed, p.w_up.scales,
+                             p.w_up.g, p.x[:m], rows=rows, threads=threads)
+        else:
+            oracle.gemv(p.w.packed, p.w.scales, p.w.g, p.x[:m], rows=rows, threads=threads)
+        dt = time.perf_counter() - t0
+        t_total += dt
+        nw = 2 if p.dual else 1
+        done_bytes += nw * rows.size * (p.k // 2 + p.k // 16) + m * p.k * 2 + m * rows.size * 2
+        calls.append(f"{p.name}@M{m}")
+    return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{len(calls)} calls of 256 consecutive output rows each, cycling over the "
+                      f"sweep's projections and M in {{1,2,4,8}} ({t_total:.1f} s)"}
+
+
+# ----------------------------------------------------------------------------------------------
+# our arm
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import nvfp4_weight_only_03_b200 as nv
+    L = nv.lib()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = synth.make(WORKLOAD)
+    bytes_of = step_bytes(wl)
+    total_step_bytes = sum(bytes_of.values())
+
+    # resident inputs
+    dw = []
+    for p in wl.projections:
+        ent = {"p": p, "W": torch.from_numpy(p.w.packed).to(dev),
+               "S": torch.from_numpy(p.w.scales).to(dev), "g": p.w.g,
+               "x": torch.from_numpy(p.x.view(np.int16)).view(torch.bfloat16).to(dev),
+               "y": torch.empty((8, p.n), dtype=torch.bfloat16, device=dev)}
+        if p.dual:
+            ent["Wu"] = torch.from_numpy(p.w_up.packed).to(dev)
+            ent["Su"] = torch.from_numpy(p.w_up.scales).to(dev)
+            ent["gu"] = p.w_up.g
+        dw.append(ent)
+    ws = nv.workspace(dev)
+    wsp, wsn = ws.data_ptr(), ws.numel()
+
+    def launches(stream_handle, x_key="x", y_key="y"):
+        """[(kind, key, fn)] for one step, raw C ABI calls with precomputed arguments."""
+        seq = []
+        for m in wl.rows:
+            for e in dw:
+                p = e["p"]
+                xp, yp = e[x_key].data_ptr(), e[y_key].data_ptr()
+                if p.dual:
+                    a = (e["W"].data_ptr(), e["S"].data_ptr(), ctypes.c_float(e["g"]),
+                         e["Wu"].data_ptr(), e["Su"].data_ptr(), ctypes.c_float(e["gu"]), xp,
+                         p.k, yp, p.n, m, p.n, p.k, wsp, wsn, stream_handle)
+                    seq.append(("nvfp4_gemv_dual", (p.name, m), L.nvfp4_gemv_dual, a))
+                else:
+                    a = (e["W"].data_ptr(), e["S"].data_ptr(), ctypes.c_float(e["g"]), xp, p.k,
+                         yp, p.n, m, p.n, p.k, wsp, wsn, stream_handle)
+                    seq.append(("nvfp4_gemv", (p.name, m), L.nvfp4_gemv, a))
+        return seq
+
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+    seq = launches(sh)
+
+    def eager_step():
+        for _, _, fn, a in seq:
+            st = fn(*a)
+            if st != 0:
+                raise RuntimeError(f"launch failed: {nv.STATUS.get(st, st)}")
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            eager_step()
+    stream.synchronize()
+
+    if args.profile_steps:
+        with torch.cuda.stream(stream):
+            for _ in range(args.profile_steps):
+                eager_step()
+        stream.synchronize()
+        return None
+
+    # one step captured as a CUDA graph, with an event pair around every launch when the
+    # installed torch can record external events inside a capture
+    try:
+        ev = [(torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True)) for _ in seq]
+    except TypeError:
+        ev = None
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        cs = torch.cuda.current_stream().cuda_stream
+        cap = launches(cs)
+        for i, (_, _, fn, a) in enumerate(cap):
+            if ev is not None:
+                ev[i][0].record()
+            st = fn(*a)
+            if ev is not None:
+                ev[i][1].record()
+            if st != 0:
+                raise RuntimeError(f"capture failed: {nv.STATUS.get(st, st)}")
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t_begin.record()
+        for _ in range(args.steps):
+            graph.replay()
+        t_end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = t_begin.elapsed_time(t_end)
+    ms = max_over_ranks(ms, world)
+    # per-launch durations: the event pairs of the last replayed step inside the timed region
+    per_launch = {}
+    timing_src = "events inside the captured step, last timed replay"
+    try:
+        if ev is None:
+            raise RuntimeError("no external events")
+        for (e0, e1), (kind, key, _, _) in zip(ev, seq):
+            per_launch[key] = (kind, e0.elapsed_time(e1) * 1e3)  # us
+    except Exception:
+        timing_src = "events around eager launches after the timed region"
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in seq]
+        with torch.cuda.stream(stream):
+            for (e0, e1), (_, _, fn, a) in zip(pairs, seq):
+                e0.record()
+                fn(*a)
+                e1.record()
+        torch.cuda.synchronize()
+        for (e0, e1), (kind, key, _, _) in zip(pairs, seq):
+            per_launch[key] = (kind, e0.elapsed_time(e1) * 1e3)
+    ms_per_step = ms / args.steps
+    value = world * total_step_bytes * args.steps / (ms * 1e-3) / 1e9
+
+    # per-kernel shares and the dominant kernel's roofline
+    by_kind = {}
+    for key, (kind, us) in per_launch.items():
+        d = by_kind.setdefault(kind, {"us": 0.0, "bytes": 0, "launches": 0})
+        d["us"] += us
+        d["bytes"] += bytes_of[key]
+        d["launches"] += 1
+    dom = max(by_kind, key=lambda k: by_kind[k]["us"])
+    d = by_kind[dom]
+    achieved = d["bytes"] / (d["us"] * 1e-6) / 1e9
+    peak, peak_src = peaks()
+    traffic = None
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": peak_src,
+                "bytes_per_launch_avg": d["bytes"] / d["launches"],
+                "avg_launch_us": round(d["us"] / d["launches"], 3),
+                "timing": timing_src,
+                "share_of_step": {k: round(v["us"] / sum(x["us"] for x in by_kind.values()), 4)
+                                  for k, v in by_kind.items()}}
+    detail = {}
+    for (name, m), (kind, us) in sorted(per_launch.items(), key=lambda t: (t[0][1], t[0][0])):
+        b = bytes_of[(name, m)]
+        detail[f"{name}@M{m}"] = {"us": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
+                                  "frac": round(b / (us * 1e-6) / 1e9 / peak, 4)}
+
+    # end to end through the public API: pinned host x in, y out, every step
+    e2e = run_e2e(args, wl, dw, ws, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(wl, args.cpu_seconds)
+
+    del graph
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4(e2m1+e4m3) x bf16 -> fp32 accumulate, bf16 out",
+            "data": "synthetic (seeded N(0,0.02) weights quantised to NVFP4, N(0,1) bf16 x)",
+            "config": {"workload": WORKLOAD_DESC, "seed": wl.seed, "rows": list(wl.rows),
+                       "bytes_per_step": total_step_bytes,
+                       "l2": "inputs 0.79 GB per M pass > 126 MB L2; no flush",
+                       "launch": "one CUDA graph per step (64 kernels), persistent grid = SMs",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roofline, "e2e": e2e, "gpu_launches": len(seq) * args.steps,
+            "clocks": clk, "per_launch": detail}
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    return line
+
+
+def run_e2e(args, wl, dw, ws, world):
+    """Same metric through the public Python API: every step copies all x (pinned host ->
+    device) and reads all y back (device -> pinned host)."""
+    import torch
+    import nvfp4_weight_only_03_b200 as nv
+    hx = {e["p"].name: torch.from_numpy(e["p"].x.view(np.int16)).view(torch.bfloat16)
+          .pin_memory() for e in dw}
+    hy = {e["p"].name: torch.empty((8, e["p"].n), dtype=torch.bfloat16).pin_memory() for e in dw}
+    dx = {e["p"].name: torch.empty_like(e["x"]) for e in dw}
+    h2d = d2h = 0
+    bytes_step = sum(step_bytes(wl).values())
+    stream = torch.cuda.current_stream()
+
+    def step():
+        nonlocal h2d, d2h
+        for m in wl.rows:
+            for e in dw:
+                p = e["p"]
+                xd = dx[p.name][:m]
+                xd.copy_(hx[p.name][:m], non_blocking=True)
+                if p.dual:
+                    y = nv.gemv_dual(e["W"], e["S"], e["g"], e["Wu"], e["Su"], e["gu"], xd,
+                                     y=e["y"][:m], ws=ws)
+                else:
+                    y = nv.gemv(e["W"], e["S"], e["g"], xd, y=e["y"][:m], ws=ws)
+                hy[p.name][:m].copy_(y, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
+    for m in wl.rows:
+        for e in dw:
+            h2d += m * e["p"].k * 2
+            d2h += m * e["p"].n * 2
+    return {"value": round(world * bytes_step * args.e2e_steps / (ms * 1e-3) / 1e9, 1),
+            "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": args.e2e_steps, "api": "nvfp4_weight_only_03_b200.gemv / gemv_dual"}
+
+
+# ----------------------------------------------------------------------------------------------
+# reference arm: the CPU oracle on a bounded sample of the same workload
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    wl = synth.make(WORKLOAD)
+    import oracle
+    oracle.build()
+    # each step: the oracle on a bounded slice (256 rows) of one projection, cycling
+    order = [(p, m) for m in wl.rows for p in wl.projections]
+    threads = os.cpu_count() or 1
+
+    def step(i):
+        p, m = order[i % len(order)]
+        rows = np.arange(256)
+        if p.dual:
+            oracle.gemv_dual(p.w.packed, p.w.scales, p.w.g, p.w_up.packed, p.w_up.scales,
+                             p.w_up.g, p.x[:m], rows=rows, threads=threads)
+        else:
+            oracle.gemv(p.w.packed, p.w.scales, p.w.g, p.x[:m], rows=rows, threads=threads)
+        nw = 2 if p.dual else 1
+        return nw * 256 * (p.k // 2 + p.k // 16) + m * p.k * 2 + m * 256 * 2
+
+    for i in range(args.warmup):
+        step(i)
+    steps = min(args.steps, 64)
+    t0 = time.perf_counter()
+    b = sum(step(i) for i in range(steps))
+    dt = time.perf_counter() - t0
+    v = b / dt / 1e9
+    return {"metric": METRIC, "value": round(v, 3), "unit": "GB/s", "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": round(dt / steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD_DESC, "seed": wl.seed, "rows": list(wl.rows)},
+            "cpu_baseline": {"value": round(v, 3), "unit": "GB/s", "cores": threads,
+                             "kind": "oracle",
+                             "sample": f"each step = 256 output rows of one projection at one M, "
+                                       f"cycling over the sweep ({steps} steps, {dt:.1f} s)"},
+            "e2e": {"value": round(v, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    line = run_ours(args, world, rank, local)
+    if line is not None and rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,129 @@
+/*
+ * nvfp4.h -- C ABI of the weight-only NVFP4 GEMV library for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the weight-only 4-bit GEMV of a decoder's decode step: the kernel family
+ * the GB10 plan calls "w4a16_gemv" (w4a16_gemv_sw / w4a16_gemv_qg, single output) and
+ * "w4a16_gemv_dual" (two weight streams sharing one activation), with weights in format
+ * "nvfp4/g16" and bf16 activations ("Blueprint - circuit executor" page for
+ * qwen3.8-27b-nvfp4 on GB10, tables "Kernels the plan launches" and "Weighted nodes").
+ * Row counts 1 (plain decode) to 8 (an 8-row speculative draft/verify round, kern-qwen38-sm103
+ * model card, section "Run"; NInfer card, DFlash2 "block width 8").
+ *
+ * Storage layout (layout_version 1):
+ *   W  uint8 [N][K/2]   byte b of row n holds element k = 2b in bits 0..3 and k = 2b+1 in
+ *                       bits 4..7; each element is E2M1 (sign bit 3, exponent bits 2..1 with
+ *                       bias 1, mantissa bit 0; exponent 0 is subnormal 0.5*m).
+ *   S  uint8 [N][K/16]  one E4M3 (FN variant, bias 7, max 448) scale per 16 elements along K,
+ *                       row-major.  Scale codes must be non-negative finite (0x00..0x7E); the
+ *                       sign bit and the NaN codes 0x7F/0xFF give unspecified results.
+ *   g  float            per-tensor global scale, passed by value.
+ *   x  bf16 [M][ldx]    activations, row-major, row stride ldx elements.
+ *   y  bf16 [M][ldy]    outputs, row-major, row stride ldy elements.
+ *
+ *   y[m][n] = bf16_rn( g * sum_k E2M1(W[n][k]) * E4M3(S[n][k/16]) * x[m][k] )
+ *
+ * accumulated in fp32.  The fused dual computes, from two such weights sharing x,
+ *   o[m][n] = bf16_rn( silu(g_gate * acc_gate) * (g_up * acc_up) ),  silu(t) = t / (1 + e^-t)
+ * in fp32 -- the SiLU(gate)*up that the GB10 plan runs as a separate "moe_silu_mul" launch.
+ *
+ * Guarantees:
+ *   - Row invariance: output row m is bitwise identical for every M in 1..8 given the same
+ *     x row, weights, N, K and device (the kernel's work split depends on N, K and the SM
+ *     count, never on M).
+ *   - Determinism: identical calls give bitwise identical results.
+ *
+ * Conventions (every entry point):
+ *   - Pointers are device pointers owned by the caller; the library never allocates, frees or
+ *     synchronises.  Work is enqueued on `stream` and completes asynchronously; the buffers
+ *     must stay valid until it has run.
+ *   - Errors are returned as nvfp4_status codes (never exceptions or aborts).  Argument
+ *     checks run on the host before any CUDA call.
+ *   - The workspace (nvfp4_workspace_bytes) must be zero-filled before its first use; every
+ *     call that returns NVFP4_OK leaves it zero-filled again except for its error word (see
+ *     nvfp4_workspace_error).  Calls that may run concurrently (different streams) need
+ *     different workspaces.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cudaStream_t;
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_NULL = -1,      /* a required pointer is NULL */
+    NVFP4_ERR_SHAPE = -2,     /* N < 0, K < 0, K % 32 != 0, ldx < K, ldy < N, K too large */
+    NVFP4_ERR_ROWS = -3,      /* M < 0 or M > 8 */
+    NVFP4_ERR_ALIGN = -4,     /* pointer or stride alignment (see each call) */
+    NVFP4_ERR_ARCH = -5,      /* current device is not compute capability 10.0 (B200) */
+    NVFP4_ERR_LAUNCH = -6,    /* the CUDA launch failed (cudaGetLastError) */
+    NVFP4_ERR_WORKSPACE = -7  /* workspace NULL, misaligned or smaller than required */
+} nvfp4_status;
+
+#define NVFP4_MAX_ROWS 8
+#define NVFP4_GROUP 16
+#define NVFP4_LAYOUT_VERSION 1
+
+typedef struct {
+    int64_t n, k;
+    int64_t weight_bytes;     /* N*K/2  */
+    int64_t scale_bytes;      /* N*K/16 */
+    int64_t weight_row_bytes; /* K/2    */
+    int64_t scale_row_bytes;  /* K/16   */
+    int32_t group;            /* 16 */
+    int32_t max_rows;         /* 8 */
+    int32_t align_bytes;      /* 16: required alignment of W and x */
+    int32_t layout_version;   /* 1 */
+} nvfp4_pack_info_t;
+
+/* Sizes of the packed storage for an N x K weight (the "nvfp4/g16" format above).
+ * Pure host function.  Returns NVFP4_ERR_NULL if out is NULL, NVFP4_ERR_SHAPE if
+ * N < 0, K < 0 or K % 32 != 0. */
+int nvfp4_pack_info(int64_t n, int64_t k, nvfp4_pack_info_t* out);
+
+/* Bytes of workspace every GEMV call on the current device needs (depends only on the
+ * device's SM count).  Returns NVFP4_ERR_NULL if bytes is NULL, NVFP4_ERR_ARCH if the current
+ * device is not a B200 (no CUDA device included). */
+int nvfp4_workspace_bytes(size_t* bytes);
+
+/* y = W x (single output), see the header comment.
+ *   w, x: 16-byte aligned;  s, y: 2-byte aligned;  workspace: 16-byte aligned, at least
+ *   nvfp4_workspace_bytes() bytes, zero-filled before first use.
+ *   ldx % 8 == 0, ldx >= K;  ldy >= N.  1 <= M <= 8 (M == 0 and N == 0 are no-ops);
+ *   K % 32 == 0 (K == 0 writes zeros).
+ * Enqueued on `stream`; returns NVFP4_OK or an nvfp4_status error (nothing is enqueued on
+ * error). */
+int nvfp4_gemv(const uint8_t* w, const uint8_t* s, float global_scale, const void* x,
+               int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* workspace,
+               size_t workspace_bytes, cudaStream_t stream);
+
+/* o = silu(W_gate x) * (W_up x), fused (one pass over both weight streams), see the header
+ * comment.  Gate and up are separate pointers with their own global scales; a stacked
+ * [gate; up] buffer is passed as w_up = w_gate + N*K/2, s_up = s_gate + N*K/16.
+ * Same alignment, shape and workspace rules as nvfp4_gemv. */
+int nvfp4_gemv_dual(const uint8_t* w_gate, const uint8_t* s_gate, float global_gate,
+                    const uint8_t* w_up, const uint8_t* s_up, float global_up, const void* x,
+                    int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
+                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* The workspace's error word after the work enqueued so far has run (synchronises the
+ * stream): 0 if no kernel hit a bounded wait's limit, else a nonzero code (results of the
+ * call that set it are then invalid; zero-fill the workspace before reuse).
+ * Returns NVFP4_OK and writes *error, or an nvfp4_status error. */
+int nvfp4_workspace_error(const void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                          int32_t* error);
+
+/* Human-readable name of a status code (static string). */
+const char* nvfp4_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

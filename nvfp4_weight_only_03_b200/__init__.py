@@ -1,0 +1,179 @@
+"""Weight-only NVFP4 GEMV for NVIDIA B200 -- thin Python binding over the C ABI in include/nvfp4.h.
+
+Every step of the computation runs in the CUDA library (libnvfp4gemv.so, built in-tree for
+sm_100a).  This module only marshals torch tensors into device pointers, sizes and the current
+CUDA stream; PyTorch provides memory and streams.  There is no fallback: if the library is
+missing or the device is not a B200 the calls raise.
+
+    y = gemv(w, s, g, x)                      # y[m][n] = bf16(g * sum_k e2m1(w) e4m3(s) x)
+    o = gemv_dual(wg, sg, gg, wu, su, gu, x)  # o = bf16(silu(gate) * up)
+
+w: uint8 [N][K/2] packed e2m1 (low nibble = even k), s: uint8 [N][K/16] e4m3 scale codes,
+g: float global scale, x: bfloat16 [M][K] (M = 1..8, row stride may exceed K).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+_LIB_PATH = _build.LIB
+_lib = None
+
+STATUS = {0: "NVFP4_OK", -1: "NVFP4_ERR_NULL", -2: "NVFP4_ERR_SHAPE", -3: "NVFP4_ERR_ROWS",
+          -4: "NVFP4_ERR_ALIGN", -5: "NVFP4_ERR_ARCH", -6: "NVFP4_ERR_LAUNCH",
+          -7: "NVFP4_ERR_WORKSPACE"}
+MAX_ROWS = 8
+GROUP = 16
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class PackInfo(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int64), ("k", ctypes.c_int64),
+                ("weight_bytes", ctypes.c_int64), ("scale_bytes", ctypes.c_int64),
+                ("weight_row_bytes", ctypes.c_int64), ("scale_row_bytes", ctypes.c_int64),
+                ("group", ctypes.c_int32), ("max_rows", ctypes.c_int32),
+                ("align_bytes", ctypes.c_int32), ("layout_version", ctypes.c_int32)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """The loaded C library (ctypes).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m nvfp4_weight_only_03_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        i64, vp, c_int, sz = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.nvfp4_pack_info.argtypes = [i64, i64, ctypes.POINTER(PackInfo)]
+        L.nvfp4_workspace_bytes.argtypes = [ctypes.POINTER(sz)]
+        L.nvfp4_gemv.argtypes = [vp, vp, ctypes.c_float, vp, i64, vp, i64, c_int, i64, i64,
+                                 vp, sz, vp]
+        L.nvfp4_gemv_dual.argtypes = [vp, vp, ctypes.c_float, vp, vp, ctypes.c_float, vp, i64,
+                                      vp, i64, c_int, i64, i64, vp, sz, vp]
+        L.nvfp4_workspace_error.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
+        L.nvfp4_status_string.argtypes = [c_int]
+        L.nvfp4_status_string.restype = ctypes.c_char_p
+        for f in (L.nvfp4_pack_info, L.nvfp4_workspace_bytes, L.nvfp4_gemv, L.nvfp4_gemv_dual,
+                  L.nvfp4_workspace_error):
+            f.restype = c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise Nvfp4Error(status, where)
+
+
+def pack_info(n: int, k: int) -> dict:
+    info = PackInfo()
+    _check(lib().nvfp4_pack_info(n, k, ctypes.byref(info)), "nvfp4_pack_info")
+    return {name: getattr(info, name) for name, _ in PackInfo._fields_}
+
+
+def workspace_bytes() -> int:
+    b = ctypes.c_size_t()
+    _check(lib().nvfp4_workspace_bytes(ctypes.byref(b)), "nvfp4_workspace_bytes")
+    return int(b.value)
+
+
+_workspaces: dict = {}
+
+
+def workspace(device=None) -> torch.Tensor:
+    """A zero-filled workspace for `device` (cached; one per device, for the default use of
+    one stream at a time)."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else
+                       torch.device(device).index or 0)
+    ws = _workspaces.get(dev)
+    if ws is None:
+        with torch.cuda.device(dev):
+            ws = torch.zeros(workspace_bytes(), dtype=torch.uint8, device=dev)
+        _workspaces[dev] = ws
+    return ws
+
+
+def workspace_error(ws: torch.Tensor, stream=None) -> int:
+    err = ctypes.c_int32()
+    st = _stream(stream)
+    _check(lib().nvfp4_workspace_error(ws.data_ptr(), ws.numel(), st, ctypes.byref(err)),
+           "nvfp4_workspace_error")
+    return int(err.value)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _weight_args(w: torch.Tensor, s: torch.Tensor):
+    if w.dtype != torch.uint8 or s.dtype != torch.uint8:
+        raise TypeError("w and s must be uint8")
+    if w.dim() != 2 or s.dim() != 2 or not w.is_contiguous() or not s.is_contiguous():
+        raise ValueError("w [N][K/2] and s [N][K/16] must be contiguous 2-D tensors")
+    n, k = w.shape[0], w.shape[1] * 2
+    if s.shape[0] != n or s.shape[1] * 16 != k:
+        raise ValueError(f"scale shape {tuple(s.shape)} does not match weight {tuple(w.shape)}")
+    return n, k
+
+
+def _x_args(x: torch.Tensor, k: int):
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    if x.dim() != 2 or x.shape[1] != k or x.stride(1) != 1:
+        raise ValueError(f"x must be [M][{k}] with unit inner stride")
+    return x, x.shape[0], x.stride(0) if x.shape[0] > 1 else k
+
+
+def _out(y, m, n, x):
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    if y.dtype != torch.bfloat16 or y.dim() != 2 or y.shape != (m, n) or y.stride(1) != 1:
+        raise ValueError(f"y must be bfloat16 [{m}][{n}] with unit inner stride")
+    return y, y.stride(0) if m > 1 else n
+
+
+def gemv(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor, y: torch.Tensor = None,
+         ws: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """y[m][n] = bf16(g * sum_k e2m1(w[n][k]) * e4m3(s[n][k/16]) * x[m][k]) on the GPU."""
+    n, k = _weight_args(w, s)
+    x, m, ldx = _x_args(x, k)
+    y, ldy = _out(y, m, n, x)
+    ws = workspace(x.device) if ws is None else ws
+    st = lib().nvfp4_gemv(w.data_ptr(), s.data_ptr(), float(g), x.data_ptr(), ldx, y.data_ptr(),
+                          ldy, m, n, k, ws.data_ptr(), ws.numel(), _stream(stream))
+    _check(st, "nvfp4_gemv")
+    return y
+
+
+def gemv_dual(wg: torch.Tensor, sg: torch.Tensor, gg: float, wu: torch.Tensor, su: torch.Tensor,
+              gu: float, x: torch.Tensor, y: torch.Tensor = None, ws: torch.Tensor = None,
+              stream=None) -> torch.Tensor:
+    """o[m][n] = bf16(silu(gate) * up), gate/up the two NVFP4 GEMVs of the same x."""
+    n, k = _weight_args(wg, sg)
+    if _weight_args(wu, su) != (n, k):
+        raise ValueError("gate and up weights must have the same shape")
+    x, m, ldx = _x_args(x, k)
+    y, ldy = _out(y, m, n, x)
+    ws = workspace(x.device) if ws is None else ws
+    st = lib().nvfp4_gemv_dual(wg.data_ptr(), sg.data_ptr(), float(gg), wu.data_ptr(),
+                               su.data_ptr(), float(gu), x.data_ptr(), ldx, y.data_ptr(), ldy,
+                               m, n, k, ws.data_ptr(), ws.numel(), _stream(stream))
+    _check(st, "nvfp4_gemv_dual")
+    return y

@@ -1,0 +1,121 @@
+"""C ABI checks that need no GPU: the library loads, exports every function include/nvfp4.h
+declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from conftest import ROOT, cuda_ok
+import nvfp4_weight_only_03_b200 as nv
+from nvfp4_weight_only_03_b200 import build as nvbuild
+
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(nvfp4_\w+)\s*\(", text, re.M)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    nvbuild.build()
+    return nv.lib()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("nvfp4_pack_info", "nvfp4_gemv", "nvfp4_gemv_dual",
+                     "nvfp4_workspace_bytes", "nvfp4_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", nv.library_path()], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        getattr(L, n)  # resolvable through ctypes
+
+
+def test_library_targets_sm100a_only(L):
+    # the build flags pin the architecture; the ELF carries a CUDA fatbin section
+    assert "arch=compute_100a,code=sm_100a" in " ".join(nvbuild.NVCC_FLAGS)
+    out = subprocess.check_output(["readelf", "-S", nv.library_path()], text=True)
+    assert ".nv_fatbin" in out
+
+
+def test_pack_info():
+    info = nv.pack_info(10240, 5120)
+    assert info["weight_bytes"] == 10240 * 2560
+    assert info["scale_bytes"] == 10240 * 320
+    assert info["weight_row_bytes"] == 2560 and info["scale_row_bytes"] == 320
+    assert info["group"] == 16 and info["max_rows"] == 8
+    assert info["align_bytes"] == 16 and info["layout_version"] == 1
+    for bad in ((10, 48), (-1, 32), (4, -32)):
+        with pytest.raises(nv.Nvfp4Error) as e:
+            nv.pack_info(*bad)
+        assert e.value.status == -2
+    assert nv.lib().nvfp4_pack_info(1, 32, None) == -1
+
+
+def test_status_strings(L):
+    for code, name in nv.STATUS.items():
+        assert L.nvfp4_status_string(code).decode() == name
+    assert L.nvfp4_status_string(12345).decode() == "NVFP4_ERR_UNKNOWN"
+
+
+# Fake, never-dereferenced addresses: every case below is rejected by the host checks, which
+# run before any CUDA call, so the pointers are only inspected for alignment / NULL.
+A16 = 0x10000
+
+
+def call(L, m=1, n=64, k=64, w=A16, s=A16, x=A16, ldx=None, y=A16, ldy=None, ws=A16,
+         wsb=1 << 30):
+    ldx = k if ldx is None else ldx
+    ldy = n if ldy is None else ldy
+    return L.nvfp4_gemv(w, s, 1.0, x, ldx, y, ldy, m, n, k, ws, wsb, None)
+
+
+def call_dual(L, m=1, n=64, k=64, wu=A16, su=A16, **kw):
+    return L.nvfp4_gemv_dual(A16, A16, 1.0, wu, su, 1.0, A16, k, A16, n, m, n, k, A16, 1 << 30,
+                             None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(m=9), -3), (dict(m=-1), -3),
+    (dict(k=48), -2), (dict(k=-32), -2), (dict(n=-1), -2),
+    (dict(ldx=32), -2), (dict(ldy=10), -2),
+    (dict(w=None), -1), (dict(s=None), -1), (dict(x=None), -1), (dict(y=None), -1),
+    (dict(w=A16 + 8), -4), (dict(x=A16 + 8), -4), (dict(s=A16 + 1), -4), (dict(y=A16 + 1), -4),
+    (dict(k=64, ldx=68), -4),
+    (dict(ws=None), -7), (dict(ws=A16 + 4), -7),
+])
+def test_host_argument_checks(L, kw, status):
+    assert call(L, **kw) == status
+
+
+def test_noops_return_ok_without_cuda(L):
+    assert call(L, m=0) == 0
+    assert call(L, n=0) == 0
+    assert call(L, m=0, w=None, x=None, y=None) == 0
+
+
+def test_dual_host_checks(L):
+    assert L.nvfp4_gemv_dual(A16, A16, 1.0, None, A16, 1.0, A16, 64, A16, 64, 1, 64, 64, A16,
+                             1 << 30, None) == -1
+    assert L.nvfp4_gemv_dual(A16, A16, 1.0, A16 + 4, A16, 1.0, A16, 64, A16, 64, 1, 64, 64,
+                             A16, 1 << 30, None) == -4
+    assert L.nvfp4_gemv_dual(A16, A16, 1.0, A16, A16, 1.0, A16, 64, A16, 64, 10, 64, 64, A16,
+                             1 << 30, None) == -3
+
+
+@pytest.mark.skipif(cuda_ok(), reason="only meaningful on a host without a CUDA device")
+def test_valid_call_without_device_reports_arch(L):
+    assert call(L) == -5
+    b = ctypes.c_size_t()
+    assert L.nvfp4_workspace_bytes(ctypes.byref(b)) == -5
