@@ -38,10 +38,11 @@
  *     must stay valid until it has run.
  *   - Errors are returned as nvfp4_status codes (never exceptions or aborts).  Argument
  *     checks run on the host before any CUDA call.
- *   - The workspace (nvfp4_workspace_bytes) must be zero-filled before its first use; every
- *     call that returns NVFP4_OK leaves it zero-filled again except for its error word (see
- *     nvfp4_workspace_error).  Calls that may run concurrently (different streams) need
- *     different workspaces.
+ *   - The workspace (nvfp4_workspace_bytes) must be zero-filled before its first use.  It
+ *     holds an error word, one completion flag per CTA and fp32 partial sums; every call
+ *     that completes resets the flags to zero, so the same workspace serves any number of
+ *     calls in stream order (and CUDA-graph replays) without re-zeroing.  Calls that may run
+ *     concurrently (different streams) need different workspaces.
  */
 #ifndef NVFP4_H
 #define NVFP4_H

@@ -159,6 +159,33 @@ def tolerance(absum: np.ndarray) -> np.ndarray:
     return 2e-3 * np.asarray(absum) + 1e-6
 
 
+def bf16_rounding_interval(bits) -> tuple[np.ndarray, np.ndarray]:
+    """[lo, hi]: the reals that round (nearest) to each finite bf16 value -- halfway to its
+    neighbours on either side."""
+    b = np.asarray(bits, np.uint16)
+    o = bf16_ordinal(b)
+
+    def from_ordinal(v):
+        v = np.asarray(v, np.int64)
+        mag = np.abs(v).astype(np.uint16)
+        return np.where(v < 0, mag | 0x8000, mag).astype(np.uint16)
+
+    v = bf16_value(b)
+    lo = (v + bf16_value(from_ordinal(o - 1))) / 2
+    hi = (v + bf16_value(from_ordinal(o + 1))) / 2
+    return lo, hi
+
+
+def within_tolerance(y_bits, y_ref, absum) -> np.ndarray:
+    """The accumulation bound on the observable bf16 output: some real within
+    2e-3 * A + 1e-6 of y_ref rounds to y_bits (y_ref's distance to the rounding interval of
+    y_bits is within the tolerance)."""
+    lo, hi = bf16_rounding_interval(y_bits)
+    y_ref = np.asarray(y_ref, np.float64)
+    dist = np.maximum(np.maximum(lo - y_ref, y_ref - hi), 0.0)
+    return dist <= tolerance(absum)
+
+
 def bf16_ordinal(bits) -> np.ndarray:
     """Monotone integer image of bf16 bit patterns (adjacent values differ by 1; +0 == -0)."""
     b = np.asarray(bits, np.uint16).astype(np.int64)

@@ -122,3 +122,14 @@ def test_ulp_distance():
     a = np.array([0x3F80, 0x0000, 0x8000, 0x0001, 0x8001], np.uint16)
     b = np.array([0x3F81, 0x8000, 0x0001, 0x8001, 0x8002], np.uint16)
     assert list(oracle.bf16_ulp_distance(a, b)) == [1, 0, 1, 2, 1]
+
+
+def test_bf16_rounding_interval_and_tolerance_rule():
+    lo, hi = oracle.bf16_rounding_interval(np.array([0x3F80, 0x4492, 0x0000], np.uint16))
+    assert lo[0] == 1 - 2 ** -9 and hi[0] == 1 + 2 ** -8
+    assert lo[1] == 1164.0 and hi[1] == 1172.0      # bf16 1168, spacing 8
+    assert lo[2] == -(2.0 ** -134) and hi[2] == 2.0 ** -134
+    # a correctly rounded output passes even where |y - y_ref| exceeds 2e-3 A (|y| close to A)
+    assert oracle.within_tolerance(np.array([0x4492]), np.array([1164.0138]), np.array([1438.5]))[0]
+    assert not oracle.within_tolerance(np.array([0x4494]), np.array([1164.0138]),
+                                       np.array([1438.5]))[0]
