@@ -173,7 +173,7 @@ def cpu_oracle_sample(wl, seconds: float):
     rng = np.random.default_rng(0)
     order = [(p, m) for m in wl.rows for p in wl.projections]
     i = 0
-    while t_total < seconds and i < 4 * len(order):
+    while t_total < seconds and i < 100000:
         p, m = order[i % len(order)]
         i += 1
         rows = np.arange(0, min(p.n, 256)) + int(rng.integers(0, max(1, p.n - 256)))

@@ -8,15 +8,19 @@
 // kern-qwen38-sm103 model card, section "Run").  Formats and the ABI are described in nvfp4.h.
 //
 // Design (B200-first):
-//   * The path is HBM-bound: 0.5625 bytes per weight.  A persistent grid (a fixed number of
-//     CTAs per SM) splits the work -- units of (RB output rows x 128 k) in row-group-major
-//     order -- into equal contiguous ranges ("stream-K"), so every SM streams the same number
-//     of bytes.  Row groups cut by a range boundary are finished by the CTA holding their first
-//     block (the "owner", which reaches them last) after adding the other CTAs' fp32 partials
-//     in CTA order; partials and flags live in a caller-provided workspace.  No data atomics:
+//   * The path is HBM-bound: 0.5625 bytes per weight.  A persistent grid (one CTA per SM)
+//     splits the work -- units of (256 output rows x 128 k) in row-group-major order -- into
+//     equal contiguous ranges ("stream-K"), so every SM streams the same number of bytes.
+//     Row groups cut by a range boundary are finished by the CTA holding their first block
+//     (the "owner", which reaches them last) after adding the other CTAs' fp32 partials in
+//     CTA order; partials and flags live in a caller-provided workspace.  No data atomics:
 //     the result is deterministic and the split depends only on (N, K, SM count), never on M.
-//   * Each lane streams 16-byte chunks of two weight rows per 16-row tile with L1-bypassing
-//     loads, prefetched D units ahead in registers, plus the 2-byte pair of group scales.
+//   * A producer warp streams the packed weights with TMA (cp.async.bulk.tensor, one 256-row x
+//     64-byte box per unit and weight stream, zero-filled past N and K, no multicast) into a
+//     ring of shared-memory stages guarded by mbarriers; eight consumer warps decode and
+//     multiply.  The ring keeps up to 128 KB per SM in flight without spending registers.
+//     The e4m3 scales (1/9 of the bytes) are loaded by the consumers themselves, several
+//     units ahead.
 //   * Decode in registers with the hardware conversions: cvt e2m1x2 -> f16x2 turns each byte
 //     (two nibbles, k and k+1) into an f16 pair, cvt e4m3x2 -> f16x2 turns two scale codes into
 //     f16, and one f16x2 multiply gives A = e2m1 * e4m3, exact in f16 (at most 6 significant
@@ -25,13 +29,14 @@
 //     16 weight rows as A and x as B, padded to 8 columns (columns >= M are zero).  The same
 //     instruction sequence serves every M, so row m of the output depends only on x row m:
 //     bitwise row invariance across M = 1..8.
-//   * x is staged once per CTA in shared memory as f16.  Each x row m is scaled by a power of
-//     two 2^e(m) chosen from the row's largest magnitude in the CTA's k range (so it lands in
-//     [2^14, 2^15)); bf16 values convert exactly unless they are more than 2^31 times smaller
-//     than that maximum.  The partial sums are multiplied back by 2^-e(m) (exact) before they
-//     are combined.  The scale depends only on row m's data.
+//   * x is staged once per CTA in shared memory as f16 (cp.async, then converted in place).
+//     Each x row m is scaled by a power of two 2^e(m) chosen from the row's largest magnitude
+//     in the CTA's k range (so it lands in [2^14, 2^15)); bf16 values convert exactly unless
+//     they are more than 2^31 times smaller than that maximum.  The partial sums are
+//     multiplied back by 2^-e(m) (exact) before they are combined.
 //   * Epilogue in fp32: y = acc * g rounded to bf16; the dual computes
 //     silu(g_g acc_g) * (g_u acc_u) with expf and rounds once.
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -44,56 +49,53 @@ namespace {
 // ------------------------------------------------------------------------------------------
 // geometry
 
-constexpr int kBlockK = 128;         // k per unit (4 lanes x 32)
-constexpr int kSlotU4 = 16;          // uint4 of staged f16 x per block per row (256 B)
-constexpr int kRowPadU4 = 4;         // 64-byte pad between x rows (bank offset)
-constexpr int kMaxRowsPerUnit = 256; // largest RB of any configuration
-constexpr int kMaxCtasPerSm = 2;     // largest CTAs/SM of any configuration
-constexpr int kPartialFloats = kMaxRowsPerUnit * 8;  // one stream's partial slot
-constexpr int kSpinLimit = 1 << 22;  // bounded wait (~0.5-1 s)
+constexpr int kBlockK = 128;                                   // k per unit
+constexpr int kMaxRows = 256;                                  // tallest unit of any variant
+constexpr int kSlotU4 = 16;                                    // uint4 of x per block per row
+constexpr int kRowPadU4 = 4;                                   // 64-byte pad between x rows
+constexpr int kSmemMax = 220 * 1024;
+constexpr int kPartialFloats = kMaxRows * 8;                   // one stream's partial slot
+constexpr int kSpinLimit = 1 << 24;                            // bounded waits
 constexpr int64_t kMaxK = int64_t(1) << 24;
 
-template <bool DUAL, int WARPS, int R, int D, int MINB>
+// Launch geometry of each variant (build-time): consumer warps, 16-row tiles per warp and
+// ring stages.  A unit is kRows = warps * tiles * 16 output rows by 128 k; a stage holds its W
+// boxes and its scale codes (rows x 8 bytes per stream).
+#ifndef NVFP4_SINGLE_WARPS
+#define NVFP4_SINGLE_WARPS 16
+#define NVFP4_SINGLE_TILES 1
+#define NVFP4_SINGLE_STAGES 8
+#endif
+#ifndef NVFP4_DUAL_WARPS
+#define NVFP4_DUAL_WARPS 16
+#define NVFP4_DUAL_TILES 1
+#define NVFP4_DUAL_STAGES 4
+#endif
+template <bool DUAL, int WARPS, int TILES, int STAGES>
 struct Geo {
     static constexpr int kStreams = DUAL ? 2 : 1;
-    static constexpr int kWarps = WARPS;
-    static constexpr int kTiles = R;      // 16-row mma tiles per warp
-    static constexpr int kDepth = D;      // units prefetched ahead
-    static constexpr int kMinBlocks = MINB;
-    static constexpr int kThreads = WARPS * 32;
-    static constexpr int kRows = WARPS * R * 16;
-    static constexpr int kSmemBudget = MINB == 1 ? 200 * 1024 : 100 * 1024;
-    static_assert(kRows <= kMaxRowsPerUnit, "unit too tall for the workspace slots");
-    static_assert(MINB <= kMaxCtasPerSm, "too many CTAs per SM for the workspace");
+    static constexpr int kConsumerWarps = WARPS;
+    static constexpr int kConsumers = WARPS * 32;
+    static constexpr int kThreads = kConsumers + 32;           // + one producer warp
+    static constexpr int kTiles = TILES;                       // 16-row mma tiles per warp
+    static constexpr int kRows = WARPS * TILES * 16;           // rows per unit
+    static constexpr int kBoxBytes = kRows * (kBlockK / 2);    // W per unit and stream
+    static constexpr int kScaleBytes = kRows * (kBlockK / 16); // scales per unit and stream
+    static constexpr int kStages = STAGES;
+    static constexpr int kStageBytes = kStreams * (kBoxBytes + kScaleBytes);
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static_assert(kRows <= kMaxRows, "unit taller than a TMA box / partial slot");
 };
-
-// Launch configurations (selected at build time; the work split, and therefore the fp32
-// summation order, depends on them, never on M).
-#ifndef NVFP4_SINGLE_CFG
-#define NVFP4_SINGLE_CFG 0
-#endif
-#ifndef NVFP4_DUAL_CFG
-#define NVFP4_DUAL_CFG 0
-#endif
-#if NVFP4_SINGLE_CFG == 0
-using GeoSingle = Geo<false, 8, 2, 3, 1>;
-#elif NVFP4_SINGLE_CFG == 1
-using GeoSingle = Geo<false, 8, 1, 4, 2>;
-#elif NVFP4_SINGLE_CFG == 2
-using GeoSingle = Geo<false, 16, 1, 3, 1>;
-#else
-using GeoSingle = Geo<false, 4, 2, 4, 2>;
-#endif
-#if NVFP4_DUAL_CFG == 0
-using GeoDual = Geo<true, 8, 2, 2, 1>;
-#elif NVFP4_DUAL_CFG == 1
-using GeoDual = Geo<true, 8, 1, 3, 2>;
-#else
-using GeoDual = Geo<true, 16, 1, 2, 1>;
-#endif
+template <bool DUAL> struct CfgSel;
+template <> struct CfgSel<false> {
+    using type = Geo<false, NVFP4_SINGLE_WARPS, NVFP4_SINGLE_TILES, NVFP4_SINGLE_STAGES>;
+};
+template <> struct CfgSel<true> {
+    using type = Geo<true, NVFP4_DUAL_WARPS, NVFP4_DUAL_TILES, NVFP4_DUAL_STAGES>;
+};
+template <bool DUAL> using Cfg = typename CfgSel<DUAL>::type;
 
 struct Params {
-    const uint8_t* w[2];
     const uint8_t* s[2];
     float g[2];          // global scales
     const uint16_t* x;
@@ -114,18 +116,70 @@ struct Params {
 // ------------------------------------------------------------------------------------------
 // device helpers
 
-__device__ __forceinline__ uint4 ld_stream16(const uint8_t* p) {
-    uint4 r;
-    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-        : "l"(p));
-    return r;
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint32_t ld_scale2(const uint8_t* p) {
-    unsigned short v;
-    asm("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
-    return v;
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+
+// Bounded wait for the phase with the given parity to complete; false after the limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
+    const uint32_t a = smem_u32(b);
+    for (int it = 0; it < kSpinLimit; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void named_barrier(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async8(void* dst, const void* src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(valid ? 8 : 0)
+                 : "memory");
+}
+
+// The mbarrier receives one arrival when all of this thread's earlier cp.async have landed.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* b) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(b))
+                 : "memory");
 }
 
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
@@ -192,62 +246,29 @@ __device__ __forceinline__ uint16_t f2bf(float v) {
 
 __device__ __forceinline__ float bf2f(uint32_t b16) { return __uint_as_float(b16 << 16); }
 
-// One lane's view of one 128-k unit of one weight stream: rows g and g+8 of each tile.
-template <int R>
-struct UnitRegs {
-    uint4 wa[R], wb[R];
-    uint32_t sa[R], sb[R];
-};
-
-// Per-stream row cursor of a lane: pointers to row (group_row0 + warp*R*16 + g) at k = 32q.
-struct RowCursor {
-    const uint8_t* w;
-    const uint8_t* s;
-};
-
-template <int R>
-__device__ __forceinline__ void load_unit(UnitRegs<R>& r, const RowCursor& c, uint32_t rows_ok,
-                                          bool kok, int b, uint32_t wrow, uint32_t srow) {
+// A lane's decoded view of one stage for one stream: the multiply-ready k-step operands.
+__device__ __forceinline__ void compute_tile(float (&acc)[2][4], uint4 wa, uint4 wb, uint32_t sca,
+                                             uint32_t scb, const uint4 (&xv)[4]) {
+    const uint32_t Sa = scale_pair(sca), Sb = scale_pair(scb);
+    const uint32_t sa0 = bcast_lo(Sa), sa1 = bcast_hi(Sa);
+    const uint32_t sb0 = bcast_lo(Sb), sb1 = bcast_hi(Sb);
+    const uint32_t A[4] = {wa.x, wa.y, wa.z, wa.w};
+    const uint32_t B[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-    for (int t = 0; t < R; ++t) {
-        const bool va = kok && ((rows_ok >> (2 * t)) & 1u);
-        const bool vb = kok && ((rows_ok >> (2 * t + 1)) & 1u);
-        const uint32_t wo = (uint32_t)(16 * t) * wrow + (uint32_t)b * 64u;
-        const uint32_t so = (uint32_t)(16 * t) * srow + (uint32_t)b * 8u;
-        r.wa[t] = va ? ld_stream16(c.w + wo) : make_uint4(0, 0, 0, 0);
-        r.wb[t] = vb ? ld_stream16(c.w + wo + 8u * wrow) : make_uint4(0, 0, 0, 0);
-        r.sa[t] = va ? ld_scale2(c.s + so) : 0u;
-        r.sb[t] = vb ? ld_scale2(c.s + so + 8u * srow) : 0u;
-    }
-}
-
-// acc[t][h][i]: tile t, h = 0 for the first mma of each word (k-step A), 1 for the second.
-template <int R>
-__device__ __forceinline__ void compute_unit(float (&acc)[R][2][4], const UnitRegs<R>& r,
-                                             const uint4 (&xv)[4]) {
+    for (int j = 0; j < 4; ++j) {
+        uint32_t pa[4], pb[4];
+        decode_word(A[j], pa);
+        decode_word(B[j], pb);
+        const uint32_t sA = j < 2 ? sa0 : sa1, sB = j < 2 ? sb0 : sb1;
 #pragma unroll
-    for (int t = 0; t < R; ++t) {
-        const uint32_t Sa = scale_pair(r.sa[t]), Sb = scale_pair(r.sb[t]);
-        const uint32_t sa0 = bcast_lo(Sa), sa1 = bcast_hi(Sa);
-        const uint32_t sb0 = bcast_lo(Sb), sb1 = bcast_hi(Sb);
-        const uint32_t wa[4] = {r.wa[t].x, r.wa[t].y, r.wa[t].z, r.wa[t].w};
-        const uint32_t wb[4] = {r.wb[t].x, r.wb[t].y, r.wb[t].z, r.wb[t].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            uint32_t pa[4], pb[4];
-            decode_word(wa[j], pa);
-            decode_word(wb[j], pb);
-            const uint32_t sA = j < 2 ? sa0 : sa1, sB = j < 2 ? sb0 : sb1;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                pa[i] = hmul2(pa[i], sA);
-                pb[i] = hmul2(pb[i], sB);
-            }
-            // k-step A: logical k {2q, 2q+1 | 2q+8, 2q+9} <- word k {0, 1 | 2, 3}
-            mma16816(acc[t][0], pa[0], pb[0], pa[1], pb[1], xv[j].x, xv[j].y);
-            // k-step B: word k {4, 5 | 6, 7}
-            mma16816(acc[t][1], pa[2], pb[2], pa[3], pb[3], xv[j].z, xv[j].w);
+        for (int i = 0; i < 4; ++i) {
+            pa[i] = hmul2(pa[i], sA);
+            pb[i] = hmul2(pb[i], sB);
         }
+        // k-step A: logical k {2q, 2q+1 | 2q+8, 2q+9} <- word k {0, 1 | 2, 3}
+        mma16816(acc[0], pa[0], pb[0], pa[1], pb[1], xv[j].x, xv[j].y);
+        // k-step B: word k {4, 5 | 6, 7}
+        mma16816(acc[1], pa[2], pb[2], pa[3], pb[3], xv[j].z, xv[j].w);
     }
 }
 
@@ -267,41 +288,31 @@ __device__ __forceinline__ void store_tile(const Params& p, int64_t row0, int g,
     }
 }
 
-template <class G>
-__device__ __forceinline__ void set_cursor(RowCursor (&c)[2], uint32_t& rows_ok, const Params& p,
-                                           int64_t rg, int warp, int g, int q) {
-    constexpr int R = G::kTiles;
-    const int64_t row = rg * G::kRows + warp * R * 16 + g;
-    rows_ok = 0;
-#pragma unroll
-    for (int t = 0; t < R; ++t) {
-        if (row + 16 * t < p.n) rows_ok |= 1u << (2 * t);
-        if (row + 16 * t + 8 < p.n) rows_ok |= 1u << (2 * t + 1);
-    }
-#pragma unroll
-    for (int s = 0; s < G::kStreams; ++s) {
-        c[s].w = p.w[s] + row * (p.k >> 1) + 16 * q;
-        c[s].s = p.s[s] + row * (p.k >> 4) + 2 * q;
-    }
-}
-
 // ------------------------------------------------------------------------------------------
 // the kernel
 
-template <class G>
-__global__ void __launch_bounds__(G::kThreads, G::kMinBlocks) nvfp4_gemv_kernel(const Params p) {
-    constexpr bool DUAL = G::kStreams == 2;
-    constexpr int NS = G::kStreams;
-    constexpr int D = G::kDepth;
-    constexpr int R = G::kTiles;
-    constexpr int NT = G::kThreads;
-    extern __shared__ uint4 xsm[];
+template <bool DUAL>
+__global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
+    nvfp4_gemv_kernel(const Params p, const __grid_constant__ CUtensorMap tm0,
+                      const __grid_constant__ CUtensorMap tm1) {
+    using C = Cfg<DUAL>;
+    constexpr int NS = C::kStreams;
+    constexpr int S = C::kStages;
+    constexpr int kTiles = C::kTiles;
+    constexpr int kRows = C::kRows;
+    constexpr int kBoxBytes = C::kBoxBytes;
+    constexpr int kScaleBytes = C::kScaleBytes;
+    constexpr int kConsumerWarps = C::kConsumerWarps;
+    constexpr int kConsumers = C::kConsumers;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    // the ring starts on a 1024-byte boundary (the launch reserves the slack)
+    uint8_t* const ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint4* const xsm = reinterpret_cast<uint4*>(ring + C::kRingBytes);
+    __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S];
     __shared__ int s_amax[8];
-    __shared__ float s_scale[8], s_descale[8];
-    __shared__ int s_ok;
+    __shared__ float s_descale[8];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = lane >> 2, q = lane & 3;
     const int cta = blockIdx.x;
     const int64_t U = p.units;
     const int64_t u_begin = U * cta / p.grid;
@@ -310,225 +321,281 @@ __global__ void __launch_bounds__(G::kThreads, G::kMinBlocks) nvfp4_gemv_kernel(
     const int kb = p.kb;
     const int64_t rg0 = u_begin / kb;
     const int b0 = (int)(u_begin - rg0 * kb);
-    const int xslots = (int)((u_end - u_begin) < kb ? (u_end - u_begin) : kb);
+    const int L = (int)(u_end - u_begin);
+    const int xslots = L < kb ? L : kb;
     const int xrow = xslots * kSlotU4 + kRowPadU4;  // uint4 per staged x row
-    const uint32_t wrow = (uint32_t)(p.k >> 1), srow = (uint32_t)(p.k >> 4);
-    const bool last_ok = (int64_t)(kb - 1) * kBlockK + 32 * q < p.k;
 
-    // ---- prefetch the first D units ------------------------------------------------------
-    RowCursor pf[2];
-    uint32_t pf_rows;
-    int64_t pf_rg = rg0;
-    int pf_b = b0;
-    set_cursor<G>(pf, pf_rows, p, pf_rg, warp, g, q);
-    UnitRegs<R> buf[D][NS];
-#pragma unroll
-    for (int d = 0; d < D; ++d) {
-        const bool live = u_begin + d < u_end;
-        const bool kok = live && (pf_b != kb - 1 || last_ok);
-#pragma unroll
-        for (int s = 0; s < NS; ++s) load_unit<R>(buf[d][s], pf[s], pf_rows, kok, pf_b, wrow, srow);
-        if (live && ++pf_b == kb) {
-            pf_b = 0;
-            ++pf_rg;
-            set_cursor<G>(pf, pf_rows, p, pf_rg, warp, g, q);
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full_bar[i], 1 + 32);  // expect_tx arrival + one per producer lane
+            mbar_init(&empty_bar[i], kConsumers);
         }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-
-    // ---- stage x as f16, scaled per row by a power of two --------------------------------
     if (tid < 8) s_amax[tid] = 0;
     __syncthreads();
+
+    // ---- producer warp: the weight boxes (TMA) and scale codes (cp.async) of every unit ----
+    if (warp == kConsumerWarps) {
+        const uint32_t srow = (uint32_t)(p.k >> 4);
+        // 8-byte scale chunks need K % 128 == 0 and 8-byte aligned scale matrices
+        bool aligned8 = (p.k % kBlockK) == 0;
+#pragma unroll
+        for (int s = 0; s < NS; ++s)
+            aligned8 = aligned8 && (reinterpret_cast<uintptr_t>(p.s[s]) & 7u) == 0;
+        int64_t rg = rg0;
+        int b = b0;
+        bool ok = true;
+        for (int i = 0; i < L; ++i) {
+            const int slot = i % S;
+            if (i >= S) {
+                if (lane == 0 && ok) ok = mbar_wait(&empty_bar[slot], ((i / S) - 1) & 1);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) {
+                    if (lane == 0) atomicExch(p.error, 2);
+                    break;
+                }
+            }
+            uint8_t* dst = ring + slot * C::kStageBytes;
+            if (lane == 0) {
+                mbar_expect_tx(&full_bar[slot], NS * kBoxBytes);
+                tma_load_2d(dst, &tm0, b * (kBlockK / 2), (int)(rg * kRows), &full_bar[slot]);
+                if (DUAL)
+                    tma_load_2d(dst + kBoxBytes, &tm1, b * (kBlockK / 2), (int)(rg * kRows),
+                                &full_bar[slot]);
+            }
+            uint8_t* sdst = dst + NS * kBoxBytes;
+#pragma unroll
+            for (int s = 0; s < NS; ++s)
+                for (int r = lane; r < kRows; r += 32) {
+                    const int64_t row = rg * kRows + r;
+                    const bool vrow = row < p.n;
+                    const uint8_t* src = p.s[s] + (vrow ? row * (int64_t)srow + (int64_t)b * 8 : 0);
+                    uint8_t* d = sdst + s * kScaleBytes + r * 8;
+                    if (aligned8) {
+                        cp_async8(d, src, vrow);
+                    } else {
+                        // K % 128 != 0: scale rows are only 2-byte aligned; copy the pairs
+                        // that exist (the last block may hold fewer than 8 groups)
+                        for (int h = 0; h < 4; ++h) {
+                            const bool v = vrow && (int64_t)b * 8 + 2 * h < (int64_t)srow;
+                            *reinterpret_cast<uint16_t*>(d + 2 * h) =
+                                v ? *reinterpret_cast<const uint16_t*>(src + 2 * h) : (uint16_t)0;
+                        }
+                    }
+                }
+            if (aligned8) cp_async_arrive(&full_bar[slot]);
+            else mbar_arrive(&full_bar[slot]);
+            if (++b == kb) {
+                b = 0;
+                ++rg;
+            }
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        return;
+    }
+
+    // ---- consumers ------------------------------------------------------------------------
+    const int g = lane >> 2, q = lane & 3;
+
+    // stage x (raw bf16) for blocks b0 .. b0+xslots-1 (mod kb) with cp.async; chunk (q, j) of a
+    // block-row holds k = blk*128 + 32q + 8j .. +8, stored at position 4q + (j ^ q) so the four
+    // lanes of a row read distinct banks
     const int per_row = xslots * kSlotU4;
-    for (int mm = 0; mm < p.m; ++mm) {
-        float amax = 0.f;
-        for (int c = tid; c < per_row; c += NT) {
+    for (int mm = 0; mm < p.m; ++mm)
+        for (int c = tid; c < per_row; c += kConsumers) {
             const int slot = c >> 4, qq = (c >> 2) & 3, jj = c & 3;
             int blk = b0 + slot;
             if (blk >= kb) blk -= kb;
             const int64_t kk = (int64_t)blk * kBlockK + 32 * qq + 8 * jj;
-            if (kk < p.k) {
-                const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.x + mm * p.ldx + kk));
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            const bool valid = kk < p.k;
+            cp_async16(&xsm[mm * xrow + slot * kSlotU4 + qq * 4 + (jj ^ qq)],
+                       p.x + (valid ? mm * p.ldx + kk : 0), valid);
+        }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    named_barrier(1, kConsumers);
+    // per-row largest magnitude, then convert in place to f16 * 2^e(m)
+    for (int mm = 0; mm < p.m; ++mm) {
+        float amax = 0.f;
+        for (int c = tid; c < per_row; c += kConsumers) {
+            const uint4 v = xsm[mm * xrow + c];
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    amax = fmaxf(amax, fabsf(bf2f(w4[i] & 0xFFFFu)));
-                    amax = fmaxf(amax, fabsf(bf2f(w4[i] >> 16)));
-                }
+            for (int i = 0; i < 4; ++i) {
+                amax = fmaxf(amax, fabsf(bf2f(w4[i] & 0xFFFFu)));
+                amax = fmaxf(amax, fabsf(bf2f(w4[i] >> 16)));
             }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
         if (lane == 0 && amax > 0.f) atomicMax(&s_amax[mm], __float_as_int(amax));
     }
-    __syncthreads();
-    if (tid < 8) {
+    named_barrier(1, kConsumers);
+    for (int mm = 0; mm < p.m; ++mm) {
         // amax in [2^E, 2^(E+1)) -> scale 2^(14-E) puts it in [2^14, 2^15), inside f16's range
-        const uint32_t bits = (uint32_t)s_amax[tid];
+        const uint32_t bits = (uint32_t)s_amax[mm];
         int e = 0;
         const int E = (int)((bits >> 23) & 0xFF) - 127;
         if (bits != 0 && E < 128) e = 14 - E;
         e = e > 126 ? 126 : (e < -126 ? -126 : e);
-        s_scale[tid] = __uint_as_float((uint32_t)(e + 127) << 23);
-        s_descale[tid] = __uint_as_float((uint32_t)(127 - e) << 23);
-    }
-    __syncthreads();
-    for (int mm = 0; mm < p.m; ++mm) {
-        const float sc = s_scale[mm];
-        for (int c = tid; c < per_row; c += NT) {
-            const int slot = c >> 4, qq = (c >> 2) & 3, jj = c & 3;
-            int blk = b0 + slot;
-            if (blk >= kb) blk -= kb;
-            const int64_t kk = (int64_t)blk * kBlockK + 32 * qq + 8 * jj;
-            uint4 o = make_uint4(0, 0, 0, 0);
-            if (kk < p.k) {
-                const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.x + mm * p.ldx + kk));
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                uint32_t h[4];
+        const float sc = __uint_as_float((uint32_t)(e + 127) << 23);
+        if (tid == 0) s_descale[mm] = __uint_as_float((uint32_t)(127 - e) << 23);
+        for (int c = tid; c < per_row; c += kConsumers) {
+            uint4 v = xsm[mm * xrow + c];
+            uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const __half2 t = __floats2half2_rn(bf2f(w4[i] & 0xFFFFu) * sc,
-                                                        bf2f(w4[i] >> 16) * sc);
-                    h[i] = *reinterpret_cast<const uint32_t*>(&t);
-                }
-                o = make_uint4(h[0], h[1], h[2], h[3]);
+            for (int i = 0; i < 4; ++i) {
+                const __half2 t = __floats2half2_rn(bf2f(w4[i] & 0xFFFFu) * sc, bf2f(w4[i] >> 16) * sc);
+                w4[i] = *reinterpret_cast<const uint32_t*>(&t);
             }
-            // swizzle the 16-byte chunk so the 4 lanes of a row hit distinct banks
-            xsm[mm * xrow + slot * kSlotU4 + qq * 4 + (jj ^ qq)] = o;
+            xsm[mm * xrow + c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
     }
-    __syncthreads();
+    named_barrier(1, kConsumers);
     const float ds0 = 2 * q < p.m ? s_descale[2 * q] : 1.f;
     const float ds1 = 2 * q + 1 < p.m ? s_descale[2 * q + 1] : 1.f;
 
-    float acc[NS][R][2][4];
+    float acc[NS][kTiles][2][4];
 #pragma unroll
     for (int s = 0; s < NS; ++s)
 #pragma unroll
-        for (int t = 0; t < R; ++t)
+        for (int t = 0; t < kTiles; ++t)
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[s][t][h][i] = 0.f;
 
     float* const my_partial = p.partial + (int64_t)cta * 2 * kPartialFloats;
-    int64_t u = u_begin;
     int64_t cur_rg = rg0;
     int cur_b = b0, seg_b0 = b0;
+    bool ok = true;
 
-    while (u < u_end) {
+#pragma unroll 1
+    for (int i = 0; i < L; ++i) {
+        int slot = cur_b - b0;
+        if (slot < 0) slot += kb;
+        uint4 xv[4];
 #pragma unroll
-        for (int d = 0; d < D; ++d) {
-            if (u >= u_end) break;
-            UnitRegs<R> cur[NS];
-            {
-                const bool live = u + D < u_end;
-                const bool kok = live && (pf_b != kb - 1 || last_ok);
+        for (int j = 0; j < 4; ++j)
+            xv[j] = g < p.m ? xsm[g * xrow + slot * kSlotU4 + q * 4 + (j ^ q)]
+                            : make_uint4(0, 0, 0, 0);
+
+        // wait for the stage, read this lane's rows and scale pairs, release the stage
+        const int st = i % S;
+        if (ok && !mbar_wait(&full_bar[st], (i / S) & 1)) {
+            ok = false;
+            atomicExch(p.error, 3);
+        }
+        const uint8_t* stage = ring + st * C::kStageBytes;
+        const uint8_t* sstage = stage + NS * kBoxBytes;
+        uint4 wa[NS][kTiles], wb[NS][kTiles];
+        uint32_t sa[NS][kTiles], sb[NS][kTiles];
 #pragma unroll
-                for (int s = 0; s < NS; ++s) {
-                    cur[s] = buf[d][s];
-                    load_unit<R>(buf[d][s], pf[s], pf_rows, kok, pf_b, wrow, srow);
-                }
-                if (live && ++pf_b == kb) {
-                    pf_b = 0;
-                    ++pf_rg;
-                    set_cursor<G>(pf, pf_rows, p, pf_rg, warp, g, q);
-                }
+        for (int s = 0; s < NS; ++s)
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t) {
+                const int ra = (warp * kTiles + t) * 16 + g;
+                wa[s][t] = *reinterpret_cast<const uint4*>(stage + s * kBoxBytes + ra * 64 + 16 * q);
+                wb[s][t] = *reinterpret_cast<const uint4*>(stage + s * kBoxBytes + (ra + 8) * 64 + 16 * q);
+                sa[s][t] = *reinterpret_cast<const uint16_t*>(sstage + s * kScaleBytes + ra * 8 + 2 * q);
+                sb[s][t] = *reinterpret_cast<const uint16_t*>(sstage + s * kScaleBytes + (ra + 8) * 8 + 2 * q);
             }
-            int slot = cur_b - b0;
-            if (slot < 0) slot += kb;
-            uint4 xv[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                xv[j] = g < p.m ? xsm[g * xrow + slot * kSlotU4 + q * 4 + (j ^ q)]
-                                : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int s = 0; s < NS; ++s) compute_unit<R>(acc[s], cur[s], xv);
-            ++u;
+        mbar_arrive(&empty_bar[st]);
 
-            if (cur_b + 1 == kb || u == u_end) {
-                // ---- end of a row-group segment: blocks seg_b0 .. cur_b of row group cur_rg
-                float tot[2][R][4];
 #pragma unroll
-                for (int s = 0; s < NS; ++s)
+        for (int s = 0; s < NS; ++s)
 #pragma unroll
-                    for (int t = 0; t < R; ++t)
+            for (int t = 0; t < kTiles; ++t)
+                compute_tile(acc[s][t], wa[s][t], wb[s][t], sa[s][t], sb[s][t], xv);
+
+        if (cur_b + 1 == kb || i + 1 == L) {
+            // ---- end of a row-group segment: blocks seg_b0 .. cur_b of row group cur_rg
+            float tot[2][kTiles][4];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            tot[s][t][i] = (acc[s][t][0][i] + acc[s][t][1][i]) * ((i & 1) ? ds1 : ds0);
-                            acc[s][t][0][i] = 0.f;
-                            acc[s][t][1][i] = 0.f;
-                        }
-                if (seg_b0 > 0) {
-                    // contributor: the row group started before this CTA's range
-                    if (2 * q < p.m) {
+            for (int s = 0; s < NS; ++s)
 #pragma unroll
-                        for (int s = 0; s < NS; ++s)
+                for (int t = 0; t < kTiles; ++t)
 #pragma unroll
-                            for (int t = 0; t < R; ++t) {
-                                float* dst = my_partial + s * kPartialFloats +
-                                             ((warp * R + t) * 32 + lane) * 4;
-                                *reinterpret_cast<float4*>(dst) = make_float4(
-                                    tot[s][t][0], tot[s][t][1], tot[s][t][2], tot[s][t][3]);
-                            }
+                    for (int e = 0; e < 4; ++e) {
+                        tot[s][t][e] = (acc[s][t][0][e] + acc[s][t][1][e]) * ((e & 1) ? ds1 : ds0);
+                        acc[s][t][0][e] = 0.f;
+                        acc[s][t][1][e] = 0.f;
                     }
+            if (seg_b0 > 0) {
+                // contributor: the row group started before this CTA's range
+                if (2 * q < p.m) {
+#pragma unroll
+                    for (int s = 0; s < NS; ++s)
+#pragma unroll
+                        for (int t = 0; t < kTiles; ++t) {
+                            float* dst = my_partial + s * kPartialFloats +
+                                         ((warp * kTiles + t) * 32 + lane) * 4;
+                            *reinterpret_cast<float4*>(dst) = make_float4(
+                                tot[s][t][0], tot[s][t][1], tot[s][t][2], tot[s][t][3]);
+                        }
+                }
+                named_barrier(1, kConsumers);
+                if (tid == 0) {
                     __threadfence();
-                    __syncthreads();
-                    if (tid == 0) st_release(p.flags + cta, 1u);
-                } else {
-                    if (cur_b + 1 != kb) {
-                        // owner: the following CTAs hold the rest of this row group, each as
-                        // the first segment of its range; add their partials in CTA order
-                        for (int c2 = cta + 1; c2 < p.grid; ++c2) {
-                            if (U * c2 / p.grid >= (cur_rg + 1) * kb) break;
-                            if (tid == 0) {
-                                int it = 0;
-                                while (ld_acquire(p.flags + c2) == 0u && ++it < kSpinLimit)
-                                    __nanosleep(32);
-                                s_ok = it < kSpinLimit;
-                                if (s_ok) p.flags[c2] = 0u;
-                                else atomicExch(p.error, 1);
-                            }
-                            __syncthreads();
-                            if (s_ok && 2 * q < p.m) {
-                                const float* src = p.partial + (int64_t)c2 * 2 * kPartialFloats;
-#pragma unroll
-                                for (int s = 0; s < NS; ++s)
-#pragma unroll
-                                    for (int t = 0; t < R; ++t) {
-                                        const float4 v = ld_cg4(src + s * kPartialFloats +
-                                                                ((warp * R + t) * 32 + lane) * 4);
-                                        tot[s][t][0] += v.x;
-                                        tot[s][t][1] += v.y;
-                                        tot[s][t][2] += v.z;
-                                        tot[s][t][3] += v.w;
-                                    }
-                            }
-                            __syncthreads();
-                        }
-                    }
-#pragma unroll
-                    for (int t = 0; t < R; ++t) {
-                        const int64_t row0 = cur_rg * G::kRows + (warp * R + t) * 16;
-                        float v[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            if (DUAL) {
-                                const float a = tot[0][t][i] * p.g[0];
-                                const float b = tot[1][t][i] * p.g[1];
-                                v[i] = a / (1.0f + expf(-a)) * b;
-                            } else {
-                                v[i] = tot[0][t][i] * p.g[0];
-                            }
-                        }
-                        store_tile(p, row0, g, q, v);
-                    }
+                    st_release(p.flags + cta, 1u);
                 }
-                seg_b0 = 0;
+            } else {
+                if (cur_b + 1 != kb) {
+                    // owner: the following CTAs hold the rest of this row group, each as the
+                    // first segment of its range; wait for all of them at once, then add their
+                    // partials in CTA order
+                    int nc = 0;
+                    while (cta + 1 + nc < p.grid &&
+                           U * (cta + 1 + nc) / p.grid < (cur_rg + 1) * kb)
+                        ++nc;
+                    for (int c = tid; c < nc; c += kConsumers) {
+                        const uint32_t* f = p.flags + cta + 1 + c;
+                        int it = 0;
+                        while (ld_acquire(f) == 0u && ++it < kSpinLimit) __nanosleep(20);
+                        if (it >= kSpinLimit) atomicExch(p.error, 1);  // result invalid
+                    }
+                    named_barrier(1, kConsumers);
+                    if (2 * q < p.m) {
+                        for (int c = 0; c < nc; ++c) {
+                            const float* src = p.partial + (int64_t)(cta + 1 + c) * 2 * kPartialFloats;
+#pragma unroll
+                            for (int s = 0; s < NS; ++s)
+#pragma unroll
+                                for (int t = 0; t < kTiles; ++t) {
+                                    const float4 v = ld_cg4(src + s * kPartialFloats +
+                                                            ((warp * kTiles + t) * 32 + lane) * 4);
+                                    tot[s][t][0] += v.x;
+                                    tot[s][t][1] += v.y;
+                                    tot[s][t][2] += v.z;
+                                    tot[s][t][3] += v.w;
+                                }
+                        }
+                    }
+                    named_barrier(1, kConsumers);
+                    for (int c = tid; c < nc; c += kConsumers) p.flags[cta + 1 + c] = 0u;
+                }
+#pragma unroll
+                for (int t = 0; t < kTiles; ++t) {
+                    const int64_t row0 = cur_rg * kRows + (warp * kTiles + t) * 16;
+                    float v[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        if (DUAL) {
+                            const float a = tot[0][t][e] * p.g[0];
+                            const float b = tot[1][t][e] * p.g[1];
+                            v[e] = a / (1.0f + expf(-a)) * b;
+                        } else {
+                            v[e] = tot[0][t][e] * p.g[0];
+                        }
+                    }
+                    store_tile(p, row0, g, q, v);
+                }
             }
-            if (++cur_b == kb) {
-                cur_b = 0;
-                ++cur_rg;
-            }
+            seg_b0 = 0;
+        }
+        if (++cur_b == kb) {
+            cur_b = 0;
+            ++cur_rg;
         }
     }
 }
@@ -542,6 +609,12 @@ struct DeviceInfo {
 };
 DeviceInfo g_dev[64];
 bool g_attr_set[2][64];
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiled g_encode = nullptr;
 
 int device_info(int* dev_out, DeviceInfo** info) {
     int dev = 0;
@@ -562,6 +635,17 @@ int device_info(int* dev_out, DeviceInfo** info) {
         di.ok = (major == 10 && minor == 0) ? 1 : 0;
     }
     if (di.ok != 1) return NVFP4_ERR_ARCH;
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn) {
+            cudaGetLastError();
+            return NVFP4_ERR_ARCH;
+        }
+        g_encode = reinterpret_cast<EncodeTiled>(fn);
+    }
     *dev_out = dev;
     *info = &di;
     return NVFP4_OK;
@@ -569,12 +653,11 @@ int device_info(int* dev_out, DeviceInfo** info) {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// workspace: [error int32 | pad to 256][flags uint32[ctas] | pad to 256][partials]
+// workspace: [error int32 | pad to 256][flags uint32[sms] | pad to 256][partials]
 size_t workspace_layout(int sms, size_t* flags_off, size_t* partial_off) {
-    const size_t ctas = (size_t)sms * kMaxCtasPerSm;
     *flags_off = 256;
-    *partial_off = 256 + align_up(ctas * 4, 256);
-    return *partial_off + ctas * 2 * kPartialFloats * sizeof(float);
+    *partial_off = 256 + align_up((size_t)sms * 4, 256);
+    return *partial_off + (size_t)sms * 2 * kPartialFloats * sizeof(float);
 }
 
 bool misaligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; }
@@ -588,6 +671,7 @@ int check_common(const void* x, int64_t ldx, const void* y, int64_t ldy, int m, 
         *noop = true;
         return NVFP4_OK;
     }
+    if (n > (int64_t(1) << 31) - kMaxRows) return NVFP4_ERR_SHAPE;
     if (ldy < n) return NVFP4_ERR_SHAPE;
     if (k > 0 && ldx < k) return NVFP4_ERR_SHAPE;
     if (!y || (k > 0 && !x)) return NVFP4_ERR_NULL;
@@ -603,11 +687,25 @@ int check_weight(const uint8_t* w, const uint8_t* s) {
     return NVFP4_OK;
 }
 
-template <class G>
+// 2-D map over a [rows][k/2] byte matrix: box = 64 bytes (128 k) x box_rows rows, zero fill
+// outside, no swizzle (two 64-byte rows share a 128-byte line, so the consumers' reads of
+// rows g and g+1 fall in distinct banks).
+bool encode_weight_map(CUtensorMap* map, const uint8_t* w, int64_t rows, int64_t k, int box_rows) {
+    const cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
+    const cuuint32_t box[2] = {(cuuint32_t)(kBlockK / 2), (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(w), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool DUAL>
 int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, const void* x,
            int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws,
            size_t ws_bytes, cudaStream_t stream) {
-    constexpr bool DUAL = G::kStreams == 2;
+    using C = Cfg<DUAL>;
     int dev = 0;
     DeviceInfo* di = nullptr;
     int st = device_info(&dev, &di);
@@ -626,8 +724,9 @@ int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, co
     }
 
     if (!g_attr_set[DUAL][dev]) {
-        if (cudaFuncSetAttribute(nvfp4_gemv_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 G::kSmemBudget) != cudaSuccess) {
+        if (cudaFuncSetAttribute(nvfp4_gemv_kernel<DUAL>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) !=
+            cudaSuccess) {
             cudaGetLastError();
             return NVFP4_ERR_LAUNCH;
         }
@@ -636,18 +735,19 @@ int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, co
 
     const int kb = (int)((k + kBlockK - 1) / kBlockK);
     const size_t slot_bytes = (size_t)kSlotU4 * 16;  // 256 B of staged x per block per row
-    const int max_grid = di->sms * G::kMinBlocks;
-    // Rows per launch: the staged x (M rows x blocks of a CTA's range) must fit the shared
-    // memory budget; a range spans at most ceil(units / grid) blocks, capped at kb.  Sized for
+    const int max_grid = di->sms;
+    // Rows per launch: the ring plus the staged x (M rows x blocks of a CTA's range) must fit
+    // shared memory; a range spans at most ceil(units / grid) blocks, capped at kb.  Sized for
     // the largest M so that the work split never depends on M.
     int64_t rows_per_launch = n;
     {
         const size_t mx = NVFP4_MAX_ROWS;
-        const int64_t max_slots =
-            (int64_t)((G::kSmemBudget - mx * kRowPadU4 * 16) / (mx * slot_bytes));
+        const int64_t max_slots = (int64_t)((kSmemMax - 1024 - C::kRingBytes -
+                                             mx * kRowPadU4 * 16) /
+                                            (mx * slot_bytes));
         if (max_slots < kb) {
             const int64_t groups = (int64_t)max_grid * max_slots / kb;
-            const int64_t cap = (groups > 0 ? groups : 1) * G::kRows;
+            const int64_t cap = (groups > 0 ? groups : 1) * C::kRows;
             if (cap < rows_per_launch) rows_per_launch = cap;
         }
     }
@@ -656,12 +756,18 @@ int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, co
     for (int64_t r0 = 0; r0 < n; r0 += rows_per_launch) {
         const int64_t nn = (n - r0) < rows_per_launch ? (n - r0) : rows_per_launch;
         Params p;
+        CUtensorMap tm[2];
+        memset(tm, 0, sizeof(tm));
         for (int i = 0; i < 2; ++i) {
             const int src = DUAL ? i : 0;
-            p.w[i] = w[src] + r0 * (k / 2);
             p.s[i] = s[src] + r0 * (k / 16);
             p.g[i] = gs[src];
+            if (i == 0 || DUAL) {
+                if (!encode_weight_map(&tm[i], w[src] + r0 * (k / 2), nn, k, C::kRows))
+                    return NVFP4_ERR_LAUNCH;
+            }
         }
+        if (!DUAL) tm[1] = tm[0];
         p.x = static_cast<const uint16_t*>(x);
         p.ldx = ldx;
         p.y = static_cast<uint16_t*>(y) + r0;
@@ -670,15 +776,16 @@ int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, co
         p.n = nn;
         p.k = k;
         p.kb = kb;
-        p.units = ((nn + G::kRows - 1) / G::kRows) * kb;
+        p.units = ((nn + C::kRows - 1) / C::kRows) * kb;
         p.grid = (int)(p.units < max_grid ? p.units : max_grid);
         p.partial = reinterpret_cast<float*>(wsb + partial_off);
         p.flags = reinterpret_cast<uint32_t*>(wsb + flags_off);
         p.error = reinterpret_cast<int32_t*>(wsb);
         const int64_t max_range = (p.units + p.grid - 1) / p.grid;
         const int slots = (int)(max_range < kb ? max_range : kb);
-        const size_t smem = (size_t)m * ((size_t)slots * slot_bytes + kRowPadU4 * 16);
-        nvfp4_gemv_kernel<G><<<p.grid, G::kThreads, smem, stream>>>(p);
+        const size_t smem =
+            1024 + C::kRingBytes + (size_t)m * ((size_t)slots * slot_bytes + kRowPadU4 * 16);
+        nvfp4_gemv_kernel<DUAL><<<p.grid, C::kThreads, smem, stream>>>(p, tm[0], tm[1]);
         if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
     }
     return NVFP4_OK;
@@ -729,8 +836,8 @@ int nvfp4_gemv(const uint8_t* w, const uint8_t* s, float global_scale, const voi
     const uint8_t* ws_[1] = {w};
     const uint8_t* ss_[1] = {s};
     const float gs[1] = {global_scale};
-    return launch<GeoSingle>(ws_, ss_, gs, x, ldx, y, ldy, m, n, k, workspace, workspace_bytes,
-                             stream);
+    return launch<false>(ws_, ss_, gs, x, ldx, y, ldy, m, n, k, workspace, workspace_bytes,
+                         stream);
 }
 
 int nvfp4_gemv_dual(const uint8_t* w_gate, const uint8_t* s_gate, float global_gate,
@@ -747,8 +854,8 @@ int nvfp4_gemv_dual(const uint8_t* w_gate, const uint8_t* s_gate, float global_g
     const uint8_t* ws_[2] = {w_gate, w_up};
     const uint8_t* ss_[2] = {s_gate, s_up};
     const float gs[2] = {global_gate, global_up};
-    return launch<GeoDual>(ws_, ss_, gs, x, ldx, y, ldy, m, n, k, workspace, workspace_bytes,
-                           stream);
+    return launch<true>(ws_, ss_, gs, x, ldx, y, ldy, m, n, k, workspace, workspace_bytes,
+                        stream);
 }
 
 int nvfp4_workspace_error(const void* workspace, size_t workspace_bytes, cudaStream_t stream,
