@@ -222,6 +222,8 @@ def run_ours(args, world, rank, local):
     ws = nv.workspace(dev)
     wsp, wsn = ws.data_ptr(), ws.numel()
 
+    flags = nv.FLAG_PREFETCH_WEIGHTS  # decode step: weights are constants
+
     def launches(stream_handle, x_key="x", y_key="y"):
         """[(kind, key, fn)] for one step, raw C ABI calls with precomputed arguments."""
         seq = []
@@ -232,12 +234,12 @@ def run_ours(args, world, rank, local):
                 if p.dual:
                     a = (e["W"].data_ptr(), e["S"].data_ptr(), ctypes.c_float(e["g"]),
                          e["Wu"].data_ptr(), e["Su"].data_ptr(), ctypes.c_float(e["gu"]), xp,
-                         p.k, yp, p.n, m, p.n, p.k, wsp, wsn, stream_handle)
-                    seq.append(("nvfp4_gemv_dual", (p.name, m), L.nvfp4_gemv_dual, a))
+                         p.k, yp, p.n, m, p.n, p.k, wsp, wsn, flags, stream_handle)
+                    seq.append(("nvfp4_gemv_dual", (p.name, m), L.nvfp4_gemv_dual_ex, a))
                 else:
                     a = (e["W"].data_ptr(), e["S"].data_ptr(), ctypes.c_float(e["g"]), xp, p.k,
-                         yp, p.n, m, p.n, p.k, wsp, wsn, stream_handle)
-                    seq.append(("nvfp4_gemv", (p.name, m), L.nvfp4_gemv, a))
+                         yp, p.n, m, p.n, p.k, wsp, wsn, flags, stream_handle)
+                    seq.append(("nvfp4_gemv", (p.name, m), L.nvfp4_gemv_ex, a))
         return seq
 
     stream = torch.cuda.Stream(device=dev)
@@ -262,27 +264,37 @@ def run_ours(args, world, rank, local):
         stream.synchronize()
         return None
 
-    # one step captured as a CUDA graph, with an event pair around every launch when the
-    # installed torch can record external events inside a capture
-    try:
-        ev = [(torch.cuda.Event(enable_timing=True, external=True),
-               torch.cuda.Event(enable_timing=True, external=True)) for _ in seq]
-    except TypeError:
+    # the step as a CUDA graph (the timed region replays it), and a second capture with an
+    # event pair around every launch for the per-kernel durations (the event nodes break the
+    # launches' overlap, so those durations are for launches that run alone)
+    def capture(with_events):
         ev = None
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        cs = torch.cuda.current_stream().cuda_stream
-        cap = launches(cs)
-        for i, (_, _, fn, a) in enumerate(cap):
-            if ev is not None:
-                ev[i][0].record()
-            st = fn(*a)
-            if ev is not None:
-                ev[i][1].record()
-            if st != 0:
-                raise RuntimeError(f"capture failed: {nv.STATUS.get(st, st)}")
+        if with_events:
+            try:
+                ev = [(torch.cuda.Event(enable_timing=True, external=True),
+                       torch.cuda.Event(enable_timing=True, external=True)) for _ in seq]
+            except TypeError:
+                return None, None
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            cs = torch.cuda.current_stream().cuda_stream
+            cap = launches(cs)
+            for i, (_, _, fn, a) in enumerate(cap):
+                if ev is not None:
+                    ev[i][0].record()
+                st = fn(*a)
+                if ev is not None:
+                    ev[i][1].record()
+                if st != 0:
+                    raise RuntimeError(f"capture failed: {nv.STATUS.get(st, st)}")
+        return graph, ev
+
+    graph, _ = capture(False)
+    graph_ev, ev = capture(True)
     for _ in range(3):
         graph.replay()
+        if graph_ev is not None:
+            graph_ev.replay()
     torch.cuda.synchronize()
 
     clocks = ClockSampler(local)
@@ -298,19 +310,25 @@ def run_ours(args, world, rank, local):
         t_end.record()
     torch.cuda.synchronize()
     barrier(world)
-    clk = clocks.stop()
     ms = t_begin.elapsed_time(t_end)
     ms = max_over_ranks(ms, world)
-    # per-launch durations: the event pairs of the last replayed step inside the timed region
+    # per-launch durations: the instrumented step, replayed right after the timed region
     per_launch = {}
-    timing_src = "events inside the captured step, last timed replay"
-    try:
-        if ev is None:
-            raise RuntimeError("no external events")
-        for (e0, e1), (kind, key, _, _) in zip(ev, seq):
-            per_launch[key] = (kind, e0.elapsed_time(e1) * 1e3)  # us
-    except Exception:
-        timing_src = "events around eager launches after the timed region"
+    reps = 10
+    if ev is not None:
+        timing_src = f"events around each launch of a captured step, median of {reps} replays"
+        samples = {key: [] for (_, key, _, _) in seq}
+        for _ in range(reps):
+            with torch.cuda.stream(stream):
+                graph_ev.replay()
+            torch.cuda.synchronize()
+            for (e0, e1), (kind, key, _, _) in zip(ev, seq):
+                samples[key].append(e0.elapsed_time(e1) * 1e3)
+        for kind, key, _, _ in seq:
+            v = sorted(samples[key])
+            per_launch[key] = (kind, v[len(v) // 2])
+    else:
+        timing_src = "events around eager launches"
         pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                  for _ in seq]
         with torch.cuda.stream(stream):
@@ -321,6 +339,7 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         for (e0, e1), (kind, key, _, _) in zip(pairs, seq):
             per_launch[key] = (kind, e0.elapsed_time(e1) * 1e3)
+    clk = clocks.stop()
     ms_per_step = ms / args.steps
     value = world * total_step_bytes * args.steps / (ms * 1e-3) / 1e9
 
@@ -342,6 +361,8 @@ def run_ours(args, world, rank, local):
                 "bytes_per_launch_avg": d["bytes"] / d["launches"],
                 "avg_launch_us": round(d["us"] / d["launches"], 3),
                 "timing": timing_src,
+                "launch_us_sum_vs_step_us": round(sum(v[1] for v in per_launch.values()) /
+                                                  (ms_per_step * 1e3), 3),
                 "share_of_step": {k: round(v["us"] / sum(x["us"] for x in by_kind.values()), 4)
                                   for k, v in by_kind.items()}}
     detail = {}
@@ -357,7 +378,7 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(wl, args.cpu_seconds)
 
-    del graph
+    del graph, graph_ev
     line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -366,7 +387,8 @@ def run_ours(args, world, rank, local):
             "config": {"workload": WORKLOAD_DESC, "seed": wl.seed, "rows": list(wl.rows),
                        "bytes_per_step": total_step_bytes,
                        "l2": "inputs 0.79 GB per M pass > 126 MB L2; no flush",
-                       "launch": "one CUDA graph per step (64 kernels), persistent grid = SMs",
+                       "launch": "one CUDA graph per step (64 kernels, programmatic dependent "
+                                 "launch between them), persistent grid = SMs",
                        "parallelism": f"replicas x{world}"},
             "roofline": roofline, "e2e": e2e, "gpu_launches": len(seq) * args.steps,
             "clocks": clk, "per_launch": detail}
@@ -397,9 +419,10 @@ def run_e2e(args, wl, dw, ws, world):
                 xd.copy_(hx[p.name][:m], non_blocking=True)
                 if p.dual:
                     y = nv.gemv_dual(e["W"], e["S"], e["g"], e["Wu"], e["Su"], e["gu"], xd,
-                                     y=e["y"][:m], ws=ws)
+                                     y=e["y"][:m], ws=ws, prefetch_weights=True)
                 else:
-                    y = nv.gemv(e["W"], e["S"], e["g"], xd, y=e["y"][:m], ws=ws)
+                    y = nv.gemv(e["W"], e["S"], e["g"], xd, y=e["y"][:m], ws=ws,
+                                prefetch_weights=True)
                 hy[p.name][:m].copy_(y, non_blocking=True)
 
     for _ in range(3):

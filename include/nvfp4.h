@@ -71,6 +71,15 @@ typedef enum {
 #define NVFP4_GROUP 16
 #define NVFP4_LAYOUT_VERSION 1
 
+/* Flags of nvfp4_gemv_ex / nvfp4_gemv_dual_ex.
+ * NVFP4_FLAG_PREFETCH_WEIGHTS: launch with programmatic dependent launch so that the packed
+ *   weights and scales start streaming while the kernel enqueued before it on the stream is
+ *   still running (the decode step's chain of projections overlaps one launch's tail with the
+ *   next one's weight stream).  x, y and the workspace are still read and written only after
+ *   that earlier work has completed.  Use it only when earlier work on the stream does not
+ *   write the weights or scales of this call. */
+#define NVFP4_FLAG_PREFETCH_WEIGHTS 1u
+
 typedef struct {
     int64_t n, k;
     int64_t weight_bytes;     /* N*K/2  */
@@ -112,6 +121,17 @@ int nvfp4_gemv_dual(const uint8_t* w_gate, const uint8_t* s_gate, float global_g
                     const uint8_t* w_up, const uint8_t* s_up, float global_up, const void* x,
                     int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* nvfp4_gemv / nvfp4_gemv_dual with launch flags (NVFP4_FLAG_*; unknown bits ->
+ * NVFP4_ERR_SHAPE).  The plain entry points are these with flags = 0. */
+int nvfp4_gemv_ex(const uint8_t* w, const uint8_t* s, float global_scale, const void* x,
+                  int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
+                  void* workspace, size_t workspace_bytes, uint32_t flags, cudaStream_t stream);
+int nvfp4_gemv_dual_ex(const uint8_t* w_gate, const uint8_t* s_gate, float global_gate,
+                       const uint8_t* w_up, const uint8_t* s_up, float global_up, const void* x,
+                       int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
+                       void* workspace, size_t workspace_bytes, uint32_t flags,
+                       cudaStream_t stream);
 
 /* The workspace's error word after the work enqueued so far has run (synchronises the
  * stream): 0 if no kernel hit a bounded wait's limit, else a nonzero code (results of the

@@ -28,6 +28,7 @@ STATUS = {0: "NVFP4_OK", -1: "NVFP4_ERR_NULL", -2: "NVFP4_ERR_SHAPE", -3: "NVFP4
           -7: "NVFP4_ERR_WORKSPACE"}
 MAX_ROWS = 8
 GROUP = 16
+FLAG_PREFETCH_WEIGHTS = 1
 
 
 class Nvfp4Error(RuntimeError):
@@ -63,11 +64,15 @@ def lib():
                                  vp, sz, vp]
         L.nvfp4_gemv_dual.argtypes = [vp, vp, ctypes.c_float, vp, vp, ctypes.c_float, vp, i64,
                                       vp, i64, c_int, i64, i64, vp, sz, vp]
+        L.nvfp4_gemv_ex.argtypes = [vp, vp, ctypes.c_float, vp, i64, vp, i64, c_int, i64, i64,
+                                    vp, sz, ctypes.c_uint32, vp]
+        L.nvfp4_gemv_dual_ex.argtypes = [vp, vp, ctypes.c_float, vp, vp, ctypes.c_float, vp, i64,
+                                         vp, i64, c_int, i64, i64, vp, sz, ctypes.c_uint32, vp]
         L.nvfp4_workspace_error.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
         L.nvfp4_status_string.argtypes = [c_int]
         L.nvfp4_status_string.restype = ctypes.c_char_p
         for f in (L.nvfp4_pack_info, L.nvfp4_workspace_bytes, L.nvfp4_gemv, L.nvfp4_gemv_dual,
-                  L.nvfp4_workspace_error):
+                  L.nvfp4_gemv_ex, L.nvfp4_gemv_dual_ex, L.nvfp4_workspace_error):
             f.restype = c_int
         _lib = L
     return _lib
@@ -150,21 +155,26 @@ def _out(y, m, n, x):
 
 
 def gemv(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor, y: torch.Tensor = None,
-         ws: torch.Tensor = None, stream=None) -> torch.Tensor:
-    """y[m][n] = bf16(g * sum_k e2m1(w[n][k]) * e4m3(s[n][k/16]) * x[m][k]) on the GPU."""
+         ws: torch.Tensor = None, stream=None, prefetch_weights: bool = False) -> torch.Tensor:
+    """y[m][n] = bf16(g * sum_k e2m1(w[n][k]) * e4m3(s[n][k/16]) * x[m][k]) on the GPU.
+
+    prefetch_weights: stream w and s before earlier work on the stream has finished
+    (programmatic dependent launch); only valid when that work does not write w or s."""
     n, k = _weight_args(w, s)
     x, m, ldx = _x_args(x, k)
     y, ldy = _out(y, m, n, x)
     ws = workspace(x.device) if ws is None else ws
-    st = lib().nvfp4_gemv(w.data_ptr(), s.data_ptr(), float(g), x.data_ptr(), ldx, y.data_ptr(),
-                          ldy, m, n, k, ws.data_ptr(), ws.numel(), _stream(stream))
+    flags = FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0
+    st = lib().nvfp4_gemv_ex(w.data_ptr(), s.data_ptr(), float(g), x.data_ptr(), ldx,
+                             y.data_ptr(), ldy, m, n, k, ws.data_ptr(), ws.numel(), flags,
+                             _stream(stream))
     _check(st, "nvfp4_gemv")
     return y
 
 
 def gemv_dual(wg: torch.Tensor, sg: torch.Tensor, gg: float, wu: torch.Tensor, su: torch.Tensor,
               gu: float, x: torch.Tensor, y: torch.Tensor = None, ws: torch.Tensor = None,
-              stream=None) -> torch.Tensor:
+              stream=None, prefetch_weights: bool = False) -> torch.Tensor:
     """o[m][n] = bf16(silu(gate) * up), gate/up the two NVFP4 GEMVs of the same x."""
     n, k = _weight_args(wg, sg)
     if _weight_args(wu, su) != (n, k):
@@ -172,8 +182,9 @@ def gemv_dual(wg: torch.Tensor, sg: torch.Tensor, gg: float, wu: torch.Tensor, s
     x, m, ldx = _x_args(x, k)
     y, ldy = _out(y, m, n, x)
     ws = workspace(x.device) if ws is None else ws
-    st = lib().nvfp4_gemv_dual(wg.data_ptr(), sg.data_ptr(), float(gg), wu.data_ptr(),
-                               su.data_ptr(), float(gu), x.data_ptr(), ldx, y.data_ptr(), ldy,
-                               m, n, k, ws.data_ptr(), ws.numel(), _stream(stream))
+    flags = FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0
+    st = lib().nvfp4_gemv_dual_ex(wg.data_ptr(), sg.data_ptr(), float(gg), wu.data_ptr(),
+                                  su.data_ptr(), float(gu), x.data_ptr(), ldx, y.data_ptr(), ldy,
+                                  m, n, k, ws.data_ptr(), ws.numel(), flags, _stream(stream))
     _check(st, "nvfp4_gemv_dual")
     return y

@@ -9,18 +9,17 @@
 //
 // Design (B200-first):
 //   * The path is HBM-bound: 0.5625 bytes per weight.  A persistent grid (one CTA per SM)
-//     splits the work -- units of (256 output rows x 128 k) in row-group-major order -- into
+//     splits the work -- units of (RB output rows x 256 k) in row-group-major order -- into
 //     equal contiguous ranges ("stream-K"), so every SM streams the same number of bytes.
-//     Row groups cut by a range boundary are finished by the CTA holding their first block
+//     Row groups cut by a range boundary are finished by the CTA holding their first unit
 //     (the "owner", which reaches them last) after adding the other CTAs' fp32 partials in
 //     CTA order; partials and flags live in a caller-provided workspace.  No data atomics:
 //     the result is deterministic and the split depends only on (N, K, SM count), never on M.
-//   * A producer warp streams the packed weights with TMA (cp.async.bulk.tensor, one 256-row x
-//     64-byte box per unit and weight stream, zero-filled past N and K, no multicast) into a
-//     ring of shared-memory stages guarded by mbarriers; eight consumer warps decode and
-//     multiply.  The ring keeps up to 128 KB per SM in flight without spending registers.
-//     The e4m3 scales (1/9 of the bytes) are loaded by the consumers themselves, several
-//     units ahead.
+//   * A producer warp streams each unit with TMA (cp.async.bulk.tensor, no multicast): one
+//     RB-row x 128-byte box of packed weights per weight stream (128-byte swizzle) and, when
+//     K % 256 == 0, one RB-row x 16-byte box of scale codes (otherwise the producer copies the
+//     scale codes with cp.async).  Boxes past N or K are zero-filled.  Stages live in a ring of
+//     shared memory guarded by mbarriers; the consumer warps decode and multiply.
 //   * Decode in registers with the hardware conversions: cvt e2m1x2 -> f16x2 turns each byte
 //     (two nibbles, k and k+1) into an f16 pair, cvt e4m3x2 -> f16x2 turns two scale codes into
 //     f16, and one f16x2 multiply gives A = e2m1 * e4m3, exact in f16 (at most 6 significant
@@ -28,12 +27,16 @@
 //   * The dot products run on the tensor cores: mma.m16n8k16 (f16 in, fp32 accumulate) with
 //     16 weight rows as A and x as B, padded to 8 columns (columns >= M are zero).  The same
 //     instruction sequence serves every M, so row m of the output depends only on x row m:
-//     bitwise row invariance across M = 1..8.
+//     bitwise row invariance across M = 1..8.  Within a 16-row tile the mma's row r is weight
+//     row perm(r) (rows r and r+1 four apart), which makes the swizzled reads conflict-free.
 //   * x is staged once per CTA in shared memory as f16 (cp.async, then converted in place).
 //     Each x row m is scaled by a power of two 2^e(m) chosen from the row's largest magnitude
 //     in the CTA's k range (so it lands in [2^14, 2^15)); bf16 values convert exactly unless
 //     they are more than 2^31 times smaller than that maximum.  The partial sums are
 //     multiplied back by 2^-e(m) (exact) before they are combined.
+//   * Optional programmatic dependent launch: the weights stream in before the preceding
+//     kernel on the stream has finished; x, y and the workspace are touched only after
+//     griddepcontrol.wait.
 //   * Epilogue in fp32: y = acc * g rounded to bf16; the dual computes
 //     silu(g_g acc_g) * (g_u acc_u) with expf and rounds once.
 #include <cuda.h>
@@ -49,51 +52,58 @@ namespace {
 // ------------------------------------------------------------------------------------------
 // geometry
 
-constexpr int kBlockK = 128;                                   // k per unit
-constexpr int kMaxRows = 256;                                  // tallest unit of any variant
-constexpr int kSlotU4 = 16;                                    // uint4 of x per block per row
-constexpr int kRowPadU4 = 4;                                   // 64-byte pad between x rows
-constexpr int kSmemMax = 220 * 1024;
-constexpr int kPartialFloats = kMaxRows * 8;                   // one stream's partial slot
-constexpr int kSpinLimit = 1 << 24;                            // bounded waits
+constexpr int kBlockK = 128;                 // k per mma block (4 lanes x 32) and per x slot
+constexpr int kUnitK = 256;                  // k per unit (one stage)
+constexpr int kWRowBytes = kUnitK / 2;       // 128 bytes of packed W per row and unit
+constexpr int kSRowBytes = kUnitK / 16;      // 16 scale codes per row and unit
+constexpr int kMaxRows = 256;                // tallest unit of any variant (TMA box limit)
+constexpr int kSlotU4 = 16;                  // uint4 of x per 128-k block per row
+constexpr int kRowPadU4 = 4;                 // 64-byte pad between x rows (bank offset)
+constexpr int kSmemMax = 226 * 1024;
+constexpr int kPartialFloats = kMaxRows * 8; // one stream's partial slot
+constexpr int kSpinLimit = 1 << 24;          // bounded waits
 constexpr int64_t kMaxK = int64_t(1) << 24;
 
-// Launch geometry of each variant (build-time): consumer warps, 16-row tiles per warp and
-// ring stages.  A unit is kRows = warps * tiles * 16 output rows by 128 k; a stage holds its W
-// boxes and its scale codes (rows x 8 bytes per stream).
+// Launch geometry of each variant (build-time): consumer warps, 16-row tiles per warp, ring
+// stages.  A unit is kRows = warps * tiles * 16 output rows by 256 k; a stage holds its W boxes
+// (rows x 128 bytes per stream) followed by its scale boxes (rows x 16 bytes per stream).
 #ifndef NVFP4_SINGLE_WARPS
-#define NVFP4_SINGLE_WARPS 16
+#define NVFP4_SINGLE_WARPS 8
 #define NVFP4_SINGLE_TILES 1
-#define NVFP4_SINGLE_STAGES 8
 #endif
 #ifndef NVFP4_DUAL_WARPS
-#define NVFP4_DUAL_WARPS 16
+#define NVFP4_DUAL_WARPS 8
 #define NVFP4_DUAL_TILES 1
-#define NVFP4_DUAL_STAGES 4
 #endif
-template <bool DUAL, int WARPS, int TILES, int STAGES>
+// The ring holds 4 to 8 stages: the row split of a launch is sized with the minimum, and a
+// launch uses as many stages as its shared memory allows (the ring depth does not change
+// the arithmetic).
+constexpr int kMinStages = 4;
+constexpr int kMaxStages = 8;
+template <bool DUAL, int WARPS, int TILES>
 struct Geo {
     static constexpr int kStreams = DUAL ? 2 : 1;
     static constexpr int kConsumerWarps = WARPS;
     static constexpr int kConsumers = WARPS * 32;
     static constexpr int kThreads = kConsumers + 32;           // + one producer warp
-    static constexpr int kTiles = TILES;                       // 16-row mma tiles per warp
+    static constexpr int kTiles = TILES;
     static constexpr int kRows = WARPS * TILES * 16;           // rows per unit
-    static constexpr int kBoxBytes = kRows * (kBlockK / 2);    // W per unit and stream
-    static constexpr int kScaleBytes = kRows * (kBlockK / 16); // scales per unit and stream
-    static constexpr int kStages = STAGES;
-    static constexpr int kStageBytes = kStreams * (kBoxBytes + kScaleBytes);
-    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kWBytes = kRows * kWRowBytes;         // W box per stream
+    static constexpr int kSBytes = kRows * kSRowBytes;         // scale box per stream
+    static constexpr int kStageBytes = kStreams * (kWBytes + kSBytes);
     static_assert(kRows <= kMaxRows, "unit taller than a TMA box / partial slot");
+    static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment (swizzle)");
 };
 template <bool DUAL> struct CfgSel;
 template <> struct CfgSel<false> {
-    using type = Geo<false, NVFP4_SINGLE_WARPS, NVFP4_SINGLE_TILES, NVFP4_SINGLE_STAGES>;
+    using type = Geo<false, NVFP4_SINGLE_WARPS, NVFP4_SINGLE_TILES>;
 };
 template <> struct CfgSel<true> {
-    using type = Geo<true, NVFP4_DUAL_WARPS, NVFP4_DUAL_TILES, NVFP4_DUAL_STAGES>;
+    using type = Geo<true, NVFP4_DUAL_WARPS, NVFP4_DUAL_TILES>;
 };
 template <bool DUAL> using Cfg = typename CfgSel<DUAL>::type;
+
+enum ScaleMode { kScaleTma = 0, kScaleAsync8 = 1, kScaleScalar = 2 };
 
 struct Params {
     const uint8_t* s[2];
@@ -105,9 +115,11 @@ struct Params {
     int m;
     int64_t n;
     int64_t k;
-    int kb;              // 128-k blocks along K (last may be partial)
-    int64_t units;       // row groups * kb
+    int ku;              // 256-k units along K (the last may be partial)
+    int64_t units;       // row groups * ku
     int grid;
+    int scale_mode;
+    int stages;          // ring depth, kMinStages .. kMaxStages
     float* partial;      // [grid][2][kPartialFloats]
     uint32_t* flags;     // [grid]
     int32_t* error;
@@ -272,11 +284,24 @@ __device__ __forceinline__ void compute_tile(float (&acc)[2][4], uint4 wa, uint4
     }
 }
 
-// Write this lane's outputs of one tile: c0 (row g, col 2q), c1 (g, 2q+1), c2 (g+8, 2q),
-// c3 (g+8, 2q+1).
-__device__ __forceinline__ void store_tile(const Params& p, int64_t row0, int g, int q,
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Row of the 16-row tile that the mma's row r (0..15) reads: rows r and r+1 of the fragment
+// are four weight rows apart, so with the 128-byte swizzle the eight lanes of a quarter-warp
+// touch eight distinct 16-byte bank groups.
+__device__ __forceinline__ int perm_row(int r) { return (r & 8) | ((r >> 1) & 3) | ((r & 1) << 2); }
+
+// Byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled box of 128-byte rows.
+__device__ __forceinline__ int swz(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
+
+// Write this lane's outputs of one tile: c0 (row ra, col 2q), c1 (ra, 2q+1), c2 (rb, 2q),
+// c3 (rb, 2q+1).
+__device__ __forceinline__ void store_tile(const Params& p, int64_t ra, int64_t rb, int q,
                                            const float (&v)[4]) {
-    const int64_t ra = row0 + g, rb = ra + 8;
     const int c0 = 2 * q, c1 = 2 * q + 1;
     if (c0 < p.m) {
         if (ra < p.n) p.y[c0 * p.ldy + ra] = f2bf(v[0]);
@@ -293,41 +318,47 @@ __device__ __forceinline__ void store_tile(const Params& p, int64_t row0, int g,
 
 template <bool DUAL>
 __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
-    nvfp4_gemv_kernel(const Params p, const __grid_constant__ CUtensorMap tm0,
-                      const __grid_constant__ CUtensorMap tm1) {
+    nvfp4_gemv_kernel(const Params p, const __grid_constant__ CUtensorMap tw0,
+                      const __grid_constant__ CUtensorMap tw1,
+                      const __grid_constant__ CUtensorMap ts0,
+                      const __grid_constant__ CUtensorMap ts1) {
     using C = Cfg<DUAL>;
     constexpr int NS = C::kStreams;
-    constexpr int S = C::kStages;
+    const int S = p.stages;
     constexpr int kTiles = C::kTiles;
     constexpr int kRows = C::kRows;
-    constexpr int kBoxBytes = C::kBoxBytes;
-    constexpr int kScaleBytes = C::kScaleBytes;
+    constexpr int kWBytes = C::kWBytes;
+    constexpr int kSBytes = C::kSBytes;
     constexpr int kConsumerWarps = C::kConsumerWarps;
     constexpr int kConsumers = C::kConsumers;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // the ring starts on a 1024-byte boundary (the launch reserves the slack)
     uint8_t* const ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint4* const xsm = reinterpret_cast<uint4*>(ring + C::kRingBytes);
-    __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S];
+    uint4* const xsm = reinterpret_cast<uint4*>(ring + S * C::kStageBytes);
+    __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages];
     __shared__ int s_amax[8];
     __shared__ float s_descale[8];
 
+    pdl_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int cta = blockIdx.x;
     const int64_t U = p.units;
     const int64_t u_begin = U * cta / p.grid;
     const int64_t u_end = U * (cta + 1) / p.grid;
     if (u_begin >= u_end) return;
-    const int kb = p.kb;
-    const int64_t rg0 = u_begin / kb;
-    const int b0 = (int)(u_begin - rg0 * kb);
+    const int ku = p.ku;
+    const int64_t rg0 = u_begin / ku;
+    const int b0 = (int)(u_begin - rg0 * ku);
     const int L = (int)(u_end - u_begin);
-    const int xslots = L < kb ? L : kb;
-    const int xrow = xslots * kSlotU4 + kRowPadU4;  // uint4 per staged x row
+    const int uslots = L < ku ? L : ku;              // distinct 256-k units of the range
+    const int xrow = 2 * uslots * kSlotU4 + kRowPadU4;  // uint4 per staged x row
 
     if (tid == 0) {
-        for (int i = 0; i < S; ++i) {
-            mbar_init(&full_bar[i], 1 + 32);  // expect_tx arrival + one per producer lane
+        // full: the expect_tx arrival, plus one per producer lane when the producer copies
+        // the scale codes itself
+        const uint32_t full_count = p.scale_mode == kScaleTma ? 1 : 1 + 32;
+        for (int i = 0; i < kMaxStages; ++i) {
+            mbar_init(&full_bar[i], full_count);
             mbar_init(&empty_bar[i], kConsumers);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -335,21 +366,21 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
     if (tid < 8) s_amax[tid] = 0;
     __syncthreads();
 
-    // ---- producer warp: the weight boxes (TMA) and scale codes (cp.async) of every unit ----
+    // ---- producer warp: stream the weight boxes and scale codes of every unit -------------
+    // (weights and scales are not written by earlier work on the stream, so this may run
+    // before griddepcontrol.wait)
     if (warp == kConsumerWarps) {
-        const uint32_t srow = (uint32_t)(p.k >> 4);
-        // 8-byte scale chunks need K % 128 == 0 and 8-byte aligned scale matrices
-        bool aligned8 = (p.k % kBlockK) == 0;
-#pragma unroll
-        for (int s = 0; s < NS; ++s)
-            aligned8 = aligned8 && (reinterpret_cast<uintptr_t>(p.s[s]) & 7u) == 0;
+        const int mode = p.scale_mode;
+        const uint32_t tx = NS * kWBytes + (mode == kScaleTma ? NS * kSBytes : 0);
+        const int64_t srow = p.k >> 4;
         int64_t rg = rg0;
         int b = b0;
         bool ok = true;
+        int slot = 0;
+        uint32_t phase = 0;  // parity of the ring pass in progress
         for (int i = 0; i < L; ++i) {
-            const int slot = i % S;
             if (i >= S) {
-                if (lane == 0 && ok) ok = mbar_wait(&empty_bar[slot], ((i / S) - 1) & 1);
+                if (lane == 0 && ok) ok = mbar_wait(&empty_bar[slot], phase ^ 1u);
                 ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
                 if (!ok) {
                     if (lane == 0) atomicExch(p.error, 2);
@@ -357,38 +388,50 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
                 }
             }
             uint8_t* dst = ring + slot * C::kStageBytes;
+            uint8_t* sdst = dst + NS * kWBytes;
+            const int y = (int)(rg * kRows);
             if (lane == 0) {
-                mbar_expect_tx(&full_bar[slot], NS * kBoxBytes);
-                tma_load_2d(dst, &tm0, b * (kBlockK / 2), (int)(rg * kRows), &full_bar[slot]);
-                if (DUAL)
-                    tma_load_2d(dst + kBoxBytes, &tm1, b * (kBlockK / 2), (int)(rg * kRows),
-                                &full_bar[slot]);
+                mbar_expect_tx(&full_bar[slot], tx);
+                tma_load_2d(dst, &tw0, b * kWRowBytes, y, &full_bar[slot]);
+                if (DUAL) tma_load_2d(dst + kWBytes, &tw1, b * kWRowBytes, y, &full_bar[slot]);
+                if (mode == kScaleTma) {
+                    tma_load_2d(sdst, &ts0, b * kSRowBytes, y, &full_bar[slot]);
+                    if (DUAL) tma_load_2d(sdst + kSBytes, &ts1, b * kSRowBytes, y, &full_bar[slot]);
+                }
             }
-            uint8_t* sdst = dst + NS * kBoxBytes;
+            if (mode != kScaleTma) {
+                // the 16 scale codes of each row for this unit (fewer in a ragged last unit)
 #pragma unroll
-            for (int s = 0; s < NS; ++s)
-                for (int r = lane; r < kRows; r += 32) {
-                    const int64_t row = rg * kRows + r;
-                    const bool vrow = row < p.n;
-                    const uint8_t* src = p.s[s] + (vrow ? row * (int64_t)srow + (int64_t)b * 8 : 0);
-                    uint8_t* d = sdst + s * kScaleBytes + r * 8;
-                    if (aligned8) {
-                        cp_async8(d, src, vrow);
-                    } else {
-                        // K % 128 != 0: scale rows are only 2-byte aligned; copy the pairs
-                        // that exist (the last block may hold fewer than 8 groups)
-                        for (int h = 0; h < 4; ++h) {
-                            const bool v = vrow && (int64_t)b * 8 + 2 * h < (int64_t)srow;
-                            *reinterpret_cast<uint16_t*>(d + 2 * h) =
-                                v ? *reinterpret_cast<const uint16_t*>(src + 2 * h) : (uint16_t)0;
+                for (int s = 0; s < NS; ++s)
+                    for (int r = lane; r < kRows; r += 32) {
+                        const int64_t row = (int64_t)y + r;
+                        const bool vrow = row < p.n;
+                        const uint8_t* src = p.s[s] + (vrow ? row * srow : 0);
+                        uint8_t* d = sdst + s * kSBytes + r * kSRowBytes;
+                        const int64_t g0 = (int64_t)b * kSRowBytes;
+                        if (mode == kScaleAsync8) {
+                            cp_async8(d, src + (vrow ? g0 : 0), vrow && g0 < srow);
+                            cp_async8(d + 8, src + (vrow && g0 + 8 < srow ? g0 + 8 : 0),
+                                      vrow && g0 + 8 < srow);
+                        } else {
+                            for (int h = 0; h < 8; ++h) {
+                                const bool v = vrow && g0 + 2 * h < srow;
+                                *reinterpret_cast<uint16_t*>(d + 2 * h) =
+                                    v ? *reinterpret_cast<const uint16_t*>(src + g0 + 2 * h)
+                                      : (uint16_t)0;
+                            }
                         }
                     }
-                }
-            if (aligned8) cp_async_arrive(&full_bar[slot]);
-            else mbar_arrive(&full_bar[slot]);
-            if (++b == kb) {
+                if (mode == kScaleAsync8) cp_async_arrive(&full_bar[slot]);
+                else mbar_arrive(&full_bar[slot]);
+            }
+            if (++b == ku) {
                 b = 0;
                 ++rg;
+            }
+            if (++slot == S) {
+                slot = 0;
+                phase ^= 1u;
             }
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
@@ -397,19 +440,22 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
 
     // ---- consumers ------------------------------------------------------------------------
     const int g = lane >> 2, q = lane & 3;
+    pdl_wait();  // x, y and the workspace may be produced / used by the preceding kernel
 
-    // stage x (raw bf16) for blocks b0 .. b0+xslots-1 (mod kb) with cp.async; chunk (q, j) of a
-    // block-row holds k = blk*128 + 32q + 8j .. +8, stored at position 4q + (j ^ q) so the four
-    // lanes of a row read distinct banks
-    const int per_row = xslots * kSlotU4;
+    // stage x (raw bf16) for the range's units (two 128-k blocks each, mod ku) with cp.async;
+    // chunk (q, j) of a block-row holds k = blk*128 + 32q + 8j .. +8, stored at position
+    // 4q + (j ^ q) so that the four lanes of a row read distinct banks
+    const int kblocks = (int)((p.k + kBlockK - 1) / kBlockK);
+    const int per_row = 2 * uslots * kSlotU4;
     for (int mm = 0; mm < p.m; ++mm)
         for (int c = tid; c < per_row; c += kConsumers) {
-            const int slot = c >> 4, qq = (c >> 2) & 3, jj = c & 3;
-            int blk = b0 + slot;
-            if (blk >= kb) blk -= kb;
+            const int xslot = c >> 4, qq = (c >> 2) & 3, jj = c & 3;
+            int ub = b0 + (xslot >> 1);
+            if (ub >= ku) ub -= ku;
+            const int blk = 2 * ub + (xslot & 1);
             const int64_t kk = (int64_t)blk * kBlockK + 32 * qq + 8 * jj;
-            const bool valid = kk < p.k;
-            cp_async16(&xsm[mm * xrow + slot * kSlotU4 + qq * 4 + (jj ^ qq)],
+            const bool valid = blk < kblocks && kk < p.k;
+            cp_async16(&xsm[mm * xrow + xslot * kSlotU4 + qq * 4 + (jj ^ qq)],
                        p.x + (valid ? mm * p.ldx + kk : 0), valid);
         }
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
@@ -455,6 +501,9 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
     const float ds0 = 2 * q < p.m ? s_descale[2 * q] : 1.f;
     const float ds1 = 2 * q + 1 < p.m ? s_descale[2 * q + 1] : 1.f;
 
+    // this lane's weight rows inside a tile (fragment rows g and g+8)
+    const int pr_a = perm_row(g), pr_b = perm_row(g + 8);
+
     float acc[NS][kTiles][2][4];
 #pragma unroll
     for (int s = 0; s < NS; ++s)
@@ -469,47 +518,51 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
     int64_t cur_rg = rg0;
     int cur_b = b0, seg_b0 = b0;
     bool ok = true;
+    int st = 0;
+    uint32_t phase = 0;
 
 #pragma unroll 1
     for (int i = 0; i < L; ++i) {
-        int slot = cur_b - b0;
-        if (slot < 0) slot += kb;
-        uint4 xv[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            xv[j] = g < p.m ? xsm[g * xrow + slot * kSlotU4 + q * 4 + (j ^ q)]
-                            : make_uint4(0, 0, 0, 0);
+        int uslot = cur_b - b0;
+        if (uslot < 0) uslot += ku;
 
-        // wait for the stage, read this lane's rows and scale pairs, release the stage
-        const int st = i % S;
-        if (ok && !mbar_wait(&full_bar[st], (i / S) & 1)) {
+        if (ok && !mbar_wait(&full_bar[st], phase)) {
             ok = false;
             atomicExch(p.error, 3);
         }
         const uint8_t* stage = ring + st * C::kStageBytes;
-        const uint8_t* sstage = stage + NS * kBoxBytes;
-        uint4 wa[NS][kTiles], wb[NS][kTiles];
-        uint32_t sa[NS][kTiles], sb[NS][kTiles];
+        const uint8_t* sstage = stage + NS * kWBytes;
 #pragma unroll
-        for (int s = 0; s < NS; ++s)
+        for (int h = 0; h < 2; ++h) {
+            // the unit's two 128-k blocks: chunks 4h .. 4h+3 of each 128-byte row
+            uint4 xv[4];
 #pragma unroll
-            for (int t = 0; t < kTiles; ++t) {
-                const int ra = (warp * kTiles + t) * 16 + g;
-                wa[s][t] = *reinterpret_cast<const uint4*>(stage + s * kBoxBytes + ra * 64 + 16 * q);
-                wb[s][t] = *reinterpret_cast<const uint4*>(stage + s * kBoxBytes + (ra + 8) * 64 + 16 * q);
-                sa[s][t] = *reinterpret_cast<const uint16_t*>(sstage + s * kScaleBytes + ra * 8 + 2 * q);
-                sb[s][t] = *reinterpret_cast<const uint16_t*>(sstage + s * kScaleBytes + (ra + 8) * 8 + 2 * q);
-            }
-        mbar_arrive(&empty_bar[st]);
+            for (int j = 0; j < 4; ++j)
+                xv[j] = g < p.m ? xsm[g * xrow + (2 * uslot + h) * kSlotU4 + q * 4 + (j ^ q)]
+                                : make_uint4(0, 0, 0, 0);
+            uint4 wa[NS][kTiles], wb[NS][kTiles];
+            uint32_t sa[NS][kTiles], sb[NS][kTiles];
+#pragma unroll
+            for (int s = 0; s < NS; ++s)
+#pragma unroll
+                for (int t = 0; t < kTiles; ++t) {
+                    const int ra = (warp * kTiles + t) * 16 + pr_a;
+                    const int rb = (warp * kTiles + t) * 16 + pr_b;
+                    wa[s][t] = *reinterpret_cast<const uint4*>(stage + s * kWBytes + swz(ra, 4 * h + q));
+                    wb[s][t] = *reinterpret_cast<const uint4*>(stage + s * kWBytes + swz(rb, 4 * h + q));
+                    sa[s][t] = *reinterpret_cast<const uint16_t*>(sstage + s * kSBytes + ra * kSRowBytes + 8 * h + 2 * q);
+                    sb[s][t] = *reinterpret_cast<const uint16_t*>(sstage + s * kSBytes + rb * kSRowBytes + 8 * h + 2 * q);
+                }
+            if (h == 1) mbar_arrive(&empty_bar[st]);
+#pragma unroll
+            for (int s = 0; s < NS; ++s)
+#pragma unroll
+                for (int t = 0; t < kTiles; ++t)
+                    compute_tile(acc[s][t], wa[s][t], wb[s][t], sa[s][t], sb[s][t], xv);
+        }
 
-#pragma unroll
-        for (int s = 0; s < NS; ++s)
-#pragma unroll
-            for (int t = 0; t < kTiles; ++t)
-                compute_tile(acc[s][t], wa[s][t], wb[s][t], sa[s][t], sb[s][t], xv);
-
-        if (cur_b + 1 == kb || i + 1 == L) {
-            // ---- end of a row-group segment: blocks seg_b0 .. cur_b of row group cur_rg
+        if (cur_b + 1 == ku || i + 1 == L) {
+            // ---- end of a row-group segment: units seg_b0 .. cur_b of row group cur_rg
             float tot[2][kTiles][4];
 #pragma unroll
             for (int s = 0; s < NS; ++s)
@@ -540,13 +593,13 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
                     st_release(p.flags + cta, 1u);
                 }
             } else {
-                if (cur_b + 1 != kb) {
+                if (cur_b + 1 != ku) {
                     // owner: the following CTAs hold the rest of this row group, each as the
                     // first segment of its range; wait for all of them at once, then add their
                     // partials in CTA order
                     int nc = 0;
                     while (cta + 1 + nc < p.grid &&
-                           U * (cta + 1 + nc) / p.grid < (cur_rg + 1) * kb)
+                           U * (cta + 1 + nc) / p.grid < (cur_rg + 1) * ku)
                         ++nc;
                     for (int c = tid; c < nc; c += kConsumers) {
                         const uint32_t* f = p.flags + cta + 1 + c;
@@ -588,14 +641,18 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
                             v[e] = tot[0][t][e] * p.g[0];
                         }
                     }
-                    store_tile(p, row0, g, q, v);
+                    store_tile(p, row0 + pr_a, row0 + pr_b, q, v);
                 }
             }
             seg_b0 = 0;
         }
-        if (++cur_b == kb) {
+        if (++cur_b == ku) {
             cur_b = 0;
             ++cur_rg;
+        }
+        if (++st == S) {
+            st = 0;
+            phase ^= 1u;
         }
     }
 }
@@ -663,8 +720,9 @@ size_t workspace_layout(int sms, size_t* flags_off, size_t* partial_off) {
 bool misaligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; }
 
 int check_common(const void* x, int64_t ldx, const void* y, int64_t ldy, int m, int64_t n,
-                 int64_t k, const void* ws, bool* noop) {
+                 int64_t k, const void* ws, uint32_t flags, bool* noop) {
     *noop = false;
+    if (flags & ~(uint32_t)NVFP4_FLAG_PREFETCH_WEIGHTS) return NVFP4_ERR_SHAPE;
     if (m < 0 || m > NVFP4_MAX_ROWS) return NVFP4_ERR_ROWS;
     if (n < 0 || k < 0 || (k % 32) != 0 || k > kMaxK) return NVFP4_ERR_SHAPE;
     if (m == 0 || n == 0) {
@@ -687,16 +745,16 @@ int check_weight(const uint8_t* w, const uint8_t* s) {
     return NVFP4_OK;
 }
 
-// 2-D map over a [rows][k/2] byte matrix: box = 64 bytes (128 k) x box_rows rows, zero fill
-// outside, no swizzle (two 64-byte rows share a 128-byte line, so the consumers' reads of
-// rows g and g+1 fall in distinct banks).
-bool encode_weight_map(CUtensorMap* map, const uint8_t* w, int64_t rows, int64_t k, int box_rows) {
-    const cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
-    const cuuint32_t box[2] = {(cuuint32_t)(kBlockK / 2), (cuuint32_t)box_rows};
+// 2-D map over a [rows][cols] byte matrix with row stride = cols: box = box_cols bytes x
+// box_rows rows, zero fill outside.
+bool encode_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t cols, int box_cols,
+                int box_rows, CUtensorMapSwizzle swizzle) {
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols};
+    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(w), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -704,8 +762,9 @@ bool encode_weight_map(CUtensorMap* map, const uint8_t* w, int64_t rows, int64_t
 template <bool DUAL>
 int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, const void* x,
            int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws,
-           size_t ws_bytes, cudaStream_t stream) {
+           size_t ws_bytes, uint32_t flags, cudaStream_t stream) {
     using C = Cfg<DUAL>;
+    constexpr int NS = C::kStreams;
     int dev = 0;
     DeviceInfo* di = nullptr;
     int st = device_info(&dev, &di);
@@ -733,20 +792,30 @@ int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, co
         g_attr_set[DUAL][dev] = true;
     }
 
-    const int kb = (int)((k + kBlockK - 1) / kBlockK);
-    const size_t slot_bytes = (size_t)kSlotU4 * 16;  // 256 B of staged x per block per row
+    // how the producer moves the scale codes: TMA needs 16-byte aligned scale rows
+    int scale_mode = kScaleTma;
+    for (int i = 0; i < NS; ++i) {
+        if ((k % kUnitK) != 0 || misaligned(s[i], 16)) scale_mode = kScaleAsync8;
+    }
+    if (scale_mode == kScaleAsync8) {
+        for (int i = 0; i < NS; ++i)
+            if ((k % kBlockK) != 0 || misaligned(s[i], 8)) scale_mode = kScaleScalar;
+    }
+
+    const int ku = (int)((k + kUnitK - 1) / kUnitK);
+    const size_t slot_bytes = (size_t)2 * kSlotU4 * 16;  // 512 B of staged x per unit per row
     const int max_grid = di->sms;
-    // Rows per launch: the ring plus the staged x (M rows x blocks of a CTA's range) must fit
-    // shared memory; a range spans at most ceil(units / grid) blocks, capped at kb.  Sized for
+    // Rows per launch: the ring plus the staged x (M rows x units of a CTA's range) must fit
+    // shared memory; a range spans at most ceil(units / grid) units, capped at ku.  Sized for
     // the largest M so that the work split never depends on M.
     int64_t rows_per_launch = n;
     {
         const size_t mx = NVFP4_MAX_ROWS;
-        const int64_t max_slots = (int64_t)((kSmemMax - 1024 - C::kRingBytes -
+        const int64_t max_slots = (int64_t)((kSmemMax - 1024 - kMinStages * C::kStageBytes -
                                              mx * kRowPadU4 * 16) /
                                             (mx * slot_bytes));
-        if (max_slots < kb) {
-            const int64_t groups = (int64_t)max_grid * max_slots / kb;
+        if (max_slots < ku) {
+            const int64_t groups = (int64_t)max_grid * max_slots / ku;
             const int64_t cap = (groups > 0 ? groups : 1) * C::kRows;
             if (cap < rows_per_launch) rows_per_launch = cap;
         }
@@ -756,18 +825,27 @@ int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, co
     for (int64_t r0 = 0; r0 < n; r0 += rows_per_launch) {
         const int64_t nn = (n - r0) < rows_per_launch ? (n - r0) : rows_per_launch;
         Params p;
-        CUtensorMap tm[2];
-        memset(tm, 0, sizeof(tm));
+        CUtensorMap tw[2], tsc[2];
+        memset(tw, 0, sizeof(tw));
+        memset(tsc, 0, sizeof(tsc));
         for (int i = 0; i < 2; ++i) {
             const int src = DUAL ? i : 0;
             p.s[i] = s[src] + r0 * (k / 16);
             p.g[i] = gs[src];
             if (i == 0 || DUAL) {
-                if (!encode_weight_map(&tm[i], w[src] + r0 * (k / 2), nn, k, C::kRows))
+                if (!encode_map(&tw[i], w[src] + r0 * (k / 2), nn, k / 2, kWRowBytes, C::kRows,
+                                CU_TENSOR_MAP_SWIZZLE_128B))
+                    return NVFP4_ERR_LAUNCH;
+                if (scale_mode == kScaleTma &&
+                    !encode_map(&tsc[i], s[src] + r0 * (k / 16), nn, k / 16, kSRowBytes, C::kRows,
+                                CU_TENSOR_MAP_SWIZZLE_NONE))
                     return NVFP4_ERR_LAUNCH;
             }
         }
-        if (!DUAL) tm[1] = tm[0];
+        if (!DUAL) {
+            tw[1] = tw[0];
+            tsc[1] = tsc[0];
+        }
         p.x = static_cast<const uint16_t*>(x);
         p.ldx = ldx;
         p.y = static_cast<uint16_t*>(y) + r0;
@@ -775,18 +853,40 @@ int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, co
         p.m = m;
         p.n = nn;
         p.k = k;
-        p.kb = kb;
-        p.units = ((nn + C::kRows - 1) / C::kRows) * kb;
+        p.ku = ku;
+        p.units = ((nn + C::kRows - 1) / C::kRows) * ku;
         p.grid = (int)(p.units < max_grid ? p.units : max_grid);
+        p.scale_mode = scale_mode;
         p.partial = reinterpret_cast<float*>(wsb + partial_off);
         p.flags = reinterpret_cast<uint32_t*>(wsb + flags_off);
         p.error = reinterpret_cast<int32_t*>(wsb);
         const int64_t max_range = (p.units + p.grid - 1) / p.grid;
-        const int slots = (int)(max_range < kb ? max_range : kb);
-        const size_t smem =
-            1024 + C::kRingBytes + (size_t)m * ((size_t)slots * slot_bytes + kRowPadU4 * 16);
-        nvfp4_gemv_kernel<DUAL><<<p.grid, C::kThreads, smem, stream>>>(p, tm[0], tm[1]);
-        if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
+        const int slots = (int)(max_range < ku ? max_range : ku);
+        const size_t xbytes = (size_t)m * ((size_t)slots * slot_bytes + kRowPadU4 * 16);
+        int stages = (int)((kSmemMax - 1024 - xbytes) / C::kStageBytes);
+        stages = stages > kMaxStages ? kMaxStages : stages;
+        if (stages < kMinStages) return NVFP4_ERR_LAUNCH;  // cannot happen: the split bounds x
+        p.stages = stages;
+        const size_t smem = 1024 + (size_t)stages * C::kStageBytes + xbytes;
+
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3(p.grid);
+        cfg.blockDim = dim3(C::kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        if (flags & NVFP4_FLAG_PREFETCH_WEIGHTS) {
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+        }
+        if (cudaLaunchKernelEx(&cfg, nvfp4_gemv_kernel<DUAL>, p, tw[0], tw[1], tsc[0], tsc[1]) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return NVFP4_ERR_LAUNCH;
+        }
     }
     return NVFP4_OK;
 }
@@ -826,26 +926,34 @@ int nvfp4_workspace_bytes(size_t* bytes) {
     return NVFP4_OK;
 }
 
-int nvfp4_gemv(const uint8_t* w, const uint8_t* s, float global_scale, const void* x,
-               int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* workspace,
-               size_t workspace_bytes, cudaStream_t stream) {
+int nvfp4_gemv_ex(const uint8_t* w, const uint8_t* s, float global_scale, const void* x,
+                  int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
+                  void* workspace, size_t workspace_bytes, uint32_t flags, cudaStream_t stream) {
     bool noop = false;
-    int st = check_common(x, ldx, y, ldy, m, n, k, workspace, &noop);
+    int st = check_common(x, ldx, y, ldy, m, n, k, workspace, flags, &noop);
     if (st != NVFP4_OK || noop) return st;
     if (k > 0 && (st = check_weight(w, s)) != NVFP4_OK) return st;
     const uint8_t* ws_[1] = {w};
     const uint8_t* ss_[1] = {s};
     const float gs[1] = {global_scale};
     return launch<false>(ws_, ss_, gs, x, ldx, y, ldy, m, n, k, workspace, workspace_bytes,
-                         stream);
+                         flags, stream);
 }
 
-int nvfp4_gemv_dual(const uint8_t* w_gate, const uint8_t* s_gate, float global_gate,
-                    const uint8_t* w_up, const uint8_t* s_up, float global_up, const void* x,
-                    int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
-                    void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+int nvfp4_gemv(const uint8_t* w, const uint8_t* s, float global_scale, const void* x,
+               int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* workspace,
+               size_t workspace_bytes, cudaStream_t stream) {
+    return nvfp4_gemv_ex(w, s, global_scale, x, ldx, y, ldy, m, n, k, workspace,
+                         workspace_bytes, 0u, stream);
+}
+
+int nvfp4_gemv_dual_ex(const uint8_t* w_gate, const uint8_t* s_gate, float global_gate,
+                       const uint8_t* w_up, const uint8_t* s_up, float global_up, const void* x,
+                       int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
+                       void* workspace, size_t workspace_bytes, uint32_t flags,
+                       cudaStream_t stream) {
     bool noop = false;
-    int st = check_common(x, ldx, y, ldy, m, n, k, workspace, &noop);
+    int st = check_common(x, ldx, y, ldy, m, n, k, workspace, flags, &noop);
     if (st != NVFP4_OK || noop) return st;
     if (k > 0) {
         if ((st = check_weight(w_gate, s_gate)) != NVFP4_OK) return st;
@@ -854,8 +962,16 @@ int nvfp4_gemv_dual(const uint8_t* w_gate, const uint8_t* s_gate, float global_g
     const uint8_t* ws_[2] = {w_gate, w_up};
     const uint8_t* ss_[2] = {s_gate, s_up};
     const float gs[2] = {global_gate, global_up};
-    return launch<true>(ws_, ss_, gs, x, ldx, y, ldy, m, n, k, workspace, workspace_bytes,
+    return launch<true>(ws_, ss_, gs, x, ldx, y, ldy, m, n, k, workspace, workspace_bytes, flags,
                         stream);
+}
+
+int nvfp4_gemv_dual(const uint8_t* w_gate, const uint8_t* s_gate, float global_gate,
+                    const uint8_t* w_up, const uint8_t* s_up, float global_up, const void* x,
+                    int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
+                    void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return nvfp4_gemv_dual_ex(w_gate, s_gate, global_gate, w_up, s_up, global_up, x, ldx, y, ldy,
+                              m, n, k, workspace, workspace_bytes, 0u, stream);
 }
 
 int nvfp4_workspace_error(const void* workspace, size_t workspace_bytes, cudaStream_t stream,

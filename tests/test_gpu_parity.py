@@ -302,3 +302,49 @@ def test_error_statuses_on_device(ws):
         nv.gemv(W, S, 1.0, x[:1], ws=ws[:100])
     torch.cuda.synchronize()
     assert nv.workspace_error(ws) == 0
+
+
+# ------------------------------------------------------------------------------------------
+# launch flags and the scale-copy paths
+
+
+def test_prefetch_flag_matches_plain_launch(ws):
+    """Programmatic dependent launch changes only when the weights stream, not the result."""
+    wl = synth.make("tiny")
+    rng = np.random.default_rng(17)
+    for n, k in ((4000, 5120), (700, 1056)):
+        w = random_weight(rng, n, k)
+        x = bf16_bits_of(rng.standard_normal((8, k)).astype(np.float32))
+        W, S, g = dev_weight(w)
+        xd = dev_x(x)
+        a = bits(nv.gemv(W, S, g, xd, ws=ws))
+        # a chain of prefetching launches on one stream, back to back
+        outs = [nv.gemv(W, S, g, xd, ws=ws, prefetch_weights=True) for _ in range(4)]
+        torch.cuda.synchronize()
+        for o in outs:
+            assert np.array_equal(bits(o), a)
+        wu = random_weight(rng, n, k)
+        Wu, Su, gu = dev_weight(wu)
+        d0 = bits(nv.gemv_dual(W, S, g, Wu, Su, gu, xd, ws=ws))
+        d1 = bits(nv.gemv_dual(W, S, g, Wu, Su, gu, xd, ws=ws, prefetch_weights=True))
+        assert np.array_equal(d0, d1)
+    assert_ws_clean(ws)
+
+
+@pytest.mark.parametrize("k,offset", [(5120, 0), (5120, 2), (5120, 8), (384, 0), (160, 0)])
+def test_scale_copy_paths(ws, k, offset):
+    """TMA scale boxes (K % 256 == 0, 16-byte aligned scales), 8-byte cp.async (K % 128 == 0,
+    8-byte aligned) and the 2-byte copy (otherwise) give identical results."""
+    rng = np.random.default_rng(k + offset)
+    n = 1000
+    w = random_weight(rng, n, k)
+    x = bf16_bits_of(rng.standard_normal((3, k)).astype(np.float32))
+    W = torch.from_numpy(w.packed).cuda()
+    buf = torch.zeros(n * (k // 16) + 64, dtype=torch.uint8, device="cuda")
+    S = buf[offset:offset + n * (k // 16)].view(n, k // 16)
+    S.copy_(torch.from_numpy(w.scales).cuda())
+    y = bits(nv.gemv(W, S, w.g, dev_x(x), ws=ws))
+    ref, a = oracle.gemv(w.packed, w.scales, w.g, x)
+    check_single(y, ref, a, f"k={k} offset={offset}")
+    y0 = bits(nv.gemv(W, torch.from_numpy(w.scales).cuda(), w.g, dev_x(x), ws=ws))
+    assert np.array_equal(y, y0)
