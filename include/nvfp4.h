@@ -133,6 +133,35 @@ int nvfp4_gemv_dual_ex(const uint8_t* w_gate, const uint8_t* s_gate, float globa
                        void* workspace, size_t workspace_bytes, uint32_t flags,
                        cudaStream_t stream);
 
+/* nvfp4_gemv for a caller that cannot provide a workspace.  The NVFP4 pages describe no such
+ * call: it is a library convenience.  It serves callers that may not allocate device memory
+ * and hold no buffer to lend: a plugin inside a host program that owns every device
+ * allocation, or a C program whose device memory is all committed before its first GEMV
+ * (cudaMalloc there would take memory outside that budget and synchronise the device).
+ *
+ * Arguments, layout, guarantees and results are those of nvfp4_gemv with flags 0; the
+ * workspace is replaced by a scratch array compiled into this library (2,622,464 bytes of
+ * device memory on each device that loads it: an error word, one flag per CTA and one pair of
+ * fp32 partial tiles per CTA, for grids of up to 160 CTAs).  The call allocates nothing.
+ *
+ * Set-up: the first call on a device (made, like every call, with that device current) looks
+ * up the array's device address with cudaGetSymbolAddress; make that first call before any
+ * stream capture.  NVFP4_ERR_LAUNCH if the lookup fails.
+ *
+ * Sharing: every call on a device uses the same array and finds it as the previous call left
+ * it.  Each call therefore first clears the error word and the flags (a cudaMemsetAsync of the
+ * first 1,024 bytes on `stream`), then launches.  Calls that overlap in time -- on different
+ * streams, or from different host threads -- race on the array and give wrong results:
+ * issue them in one stream's order.  If a bounded wait inside the kernel gives up, the kernel
+ * records it in the array's error word, which this call cannot report; callers that need
+ * that check use nvfp4_gemv with nvfp4_workspace_error.
+ *
+ * Errors: NVFP4_ERR_WORKSPACE if the device has more than 160 SMs (the array is too small:
+ * use nvfp4_gemv); otherwise those of nvfp4_gemv. */
+int nvfp4_gemv_noalloc(const uint8_t* w, const uint8_t* s, float global_scale, const void* x,
+                       int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
+                       cudaStream_t stream);
+
 /* The workspace's error word after the work enqueued so far has run (synchronises the
  * stream): 0 if no kernel hit a bounded wait's limit, else a nonzero code (results of the
  * call that set it are then invalid; zero-fill the workspace before reuse).

@@ -68,11 +68,14 @@ def lib():
                                     vp, sz, ctypes.c_uint32, vp]
         L.nvfp4_gemv_dual_ex.argtypes = [vp, vp, ctypes.c_float, vp, vp, ctypes.c_float, vp, i64,
                                          vp, i64, c_int, i64, i64, vp, sz, ctypes.c_uint32, vp]
+        L.nvfp4_gemv_noalloc.argtypes = [vp, vp, ctypes.c_float, vp, i64, vp, i64, c_int, i64,
+                                         i64, vp]
         L.nvfp4_workspace_error.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
         L.nvfp4_status_string.argtypes = [c_int]
         L.nvfp4_status_string.restype = ctypes.c_char_p
         for f in (L.nvfp4_pack_info, L.nvfp4_workspace_bytes, L.nvfp4_gemv, L.nvfp4_gemv_dual,
-                  L.nvfp4_gemv_ex, L.nvfp4_gemv_dual_ex, L.nvfp4_workspace_error):
+                  L.nvfp4_gemv_ex, L.nvfp4_gemv_dual_ex, L.nvfp4_gemv_noalloc,
+                  L.nvfp4_workspace_error):
             f.restype = c_int
         _lib = L
     return _lib
@@ -169,6 +172,20 @@ def gemv(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor, y: torch.T
                              y.data_ptr(), ldy, m, n, k, ws.data_ptr(), ws.numel(), flags,
                              _stream(stream))
     _check(st, "nvfp4_gemv")
+    return y
+
+
+def gemv_noalloc(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor,
+                 y: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """gemv through nvfp4_gemv_noalloc: the library's own scratch replaces the workspace.
+
+    Calls on one device share that scratch, so they must not overlap in time."""
+    n, k = _weight_args(w, s)
+    x, m, ldx = _x_args(x, k)
+    y, ldy = _out(y, m, n, x)
+    st = lib().nvfp4_gemv_noalloc(w.data_ptr(), s.data_ptr(), float(g), x.data_ptr(), ldx,
+                                  y.data_ptr(), ldy, m, n, k, _stream(stream))
+    _check(st, "nvfp4_gemv_noalloc")
     return y
 
 

@@ -894,6 +894,21 @@ int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, co
 }  // namespace
 
 // ------------------------------------------------------------------------------------------
+// Scratch of nvfp4_gemv_noalloc: the workspace of nvfp4_gemv (error word, one flag per CTA,
+// one pair of partial tiles per CTA, in workspace_layout's order) compiled into the library
+// for grids of up to kNoAllocSms CTAs, so that the call needs no buffer from its caller.
+
+constexpr int kNoAllocSms = 160;
+constexpr size_t kNoAllocFlagsBytes = ((size_t)kNoAllocSms * 4 + 255) / 256 * 256;
+constexpr size_t kNoAllocBytes =
+    256 + kNoAllocFlagsBytes + (size_t)kNoAllocSms * 2 * kPartialFloats * sizeof(float);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+namespace {
+void* g_noalloc_ptr[64];  // the array's device address, per device, found at the first call
+}  // namespace
+
+// ------------------------------------------------------------------------------------------
 // C ABI
 
 extern "C" {
@@ -945,6 +960,43 @@ int nvfp4_gemv(const uint8_t* w, const uint8_t* s, float global_scale, const voi
                size_t workspace_bytes, cudaStream_t stream) {
     return nvfp4_gemv_ex(w, s, global_scale, x, ldx, y, ldy, m, n, k, workspace,
                          workspace_bytes, 0u, stream);
+}
+
+int nvfp4_gemv_noalloc(const uint8_t* w, const uint8_t* s, float global_scale, const void* x,
+                       int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
+                       cudaStream_t stream) {
+    bool noop = false;
+    // check_common also vets a caller's workspace pointer; hand it a stand-in, the scratch's
+    // size is checked against the device below.
+    alignas(16) static const unsigned char stand_in[16] = {0};
+    int st = check_common(x, ldx, y, ldy, m, n, k, stand_in, 0u, &noop);
+    if (st != NVFP4_OK || noop) return st;
+    if (k > 0 && (st = check_weight(w, s)) != NVFP4_OK) return st;
+    int dev = 0;
+    DeviceInfo* di = nullptr;
+    if ((st = device_info(&dev, &di)) != NVFP4_OK) return st;
+    size_t flags_off, partial_off;
+    if (workspace_layout(di->sms, &flags_off, &partial_off) > kNoAllocBytes)
+        return NVFP4_ERR_WORKSPACE;  // more SMs than the compiled-in scratch covers
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+            cudaGetLastError();
+            return NVFP4_ERR_LAUNCH;
+        }
+        g_noalloc_ptr[dev] = ptr;
+    }
+    void* scratch = g_noalloc_ptr[dev];
+    // The previous call left its error word and flags behind; start this one from zero.
+    if (cudaMemsetAsync(scratch, 0, partial_off, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_LAUNCH;
+    }
+    const uint8_t* ws_[1] = {w};
+    const uint8_t* ss_[1] = {s};
+    const float gs[1] = {global_scale};
+    return launch<false>(ws_, ss_, gs, x, ldx, y, ldy, m, n, k, scratch, kNoAllocBytes, 0u,
+                         stream);
 }
 
 int nvfp4_gemv_dual_ex(const uint8_t* w_gate, const uint8_t* s_gate, float global_gate,

@@ -119,3 +119,12 @@ def test_valid_call_without_device_reports_arch(L):
     assert call(L) == -5
     b = ctypes.c_size_t()
     assert L.nvfp4_workspace_bytes(ctypes.byref(b)) == -5
+
+
+def test_noalloc_host_checks(L):
+    assert L.nvfp4_gemv_noalloc(A16, A16, 1.0, A16, 64, A16, 64, 9, 64, 64, None) == -3
+    assert L.nvfp4_gemv_noalloc(A16, A16, 1.0, A16 + 8, 64, A16, 64, 1, 64, 64, None) == -4
+    assert L.nvfp4_gemv_noalloc(None, A16, 1.0, A16, 64, A16, 64, 1, 64, 64, None) == -1
+    assert L.nvfp4_gemv_noalloc(A16, A16, 1.0, A16, 64, A16, 64, 0, 64, 64, None) == 0
+    if not cuda_ok():
+        assert L.nvfp4_gemv_noalloc(A16, A16, 1.0, A16, 64, A16, 64, 1, 64, 64, None) == -5
