@@ -79,6 +79,12 @@ constexpr int64_t kMaxK = int64_t(1) << 24;
 // launch uses as many stages as its shared memory allows (the ring depth does not change
 // the arithmetic).
 constexpr int kMinStages = 4;
+// Units of weights issued before the consumers have requested x (which may wait for the
+// preceding kernel): a longer queue of weight boxes ahead of those requests delays them.
+#ifndef NVFP4_PREFETCH_UNITS
+#define NVFP4_PREFETCH_UNITS 2
+#endif
+constexpr int kPrefetch = NVFP4_PREFETCH_UNITS;
 constexpr int kMaxStages = 8;
 template <bool DUAL, int WARPS, int TILES>
 struct Geo {
@@ -93,6 +99,7 @@ struct Geo {
     static constexpr int kStageBytes = kStreams * (kWBytes + kSBytes);
     static_assert(kRows <= kMaxRows, "unit taller than a TMA box / partial slot");
     static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment (swizzle)");
+    static_assert(WARPS % 8 == 0, "x staging gives each of up to 8 x rows a whole warp");
 };
 template <bool DUAL> struct CfgSel;
 template <> struct CfgSel<false> {
@@ -335,7 +342,7 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
     // the ring starts on a 1024-byte boundary (the launch reserves the slack)
     uint8_t* const ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint4* const xsm = reinterpret_cast<uint4*>(ring + S * C::kStageBytes);
-    __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages], xreq_bar;
     __shared__ int s_amax[8];
     __shared__ float s_descale[8];
 
@@ -361,6 +368,7 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
             mbar_init(&full_bar[i], full_count);
             mbar_init(&empty_bar[i], kConsumers);
         }
+        mbar_init(&xreq_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (tid < 8) s_amax[tid] = 0;
@@ -379,6 +387,16 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
         int slot = 0;
         uint32_t phase = 0;  // parity of the ring pass in progress
         for (int i = 0; i < L; ++i) {
+            if (i == kPrefetch) {
+                // the rest of the ring queues behind the consumers' requests for x, which
+                // would otherwise wait for every weight box issued before them
+                if (lane == 0 && ok) ok = mbar_wait(&xreq_bar, 0);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) {
+                    if (lane == 0) atomicExch(p.error, 2);
+                    break;
+                }
+            }
             if (i >= S) {
                 if (lane == 0 && ok) ok = mbar_wait(&empty_bar[slot], phase ^ 1u);
                 ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -458,43 +476,54 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
             cp_async16(&xsm[mm * xrow + xslot * kSlotU4 + qq * 4 + (jj ^ qq)],
                        p.x + (valid ? mm * p.ldx + kk : 0), valid);
         }
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    named_barrier(1, kConsumers);          // every consumer has issued its copies of x ...
+    if (tid == 0) mbar_arrive(&xreq_bar);  // ... so the producer may queue the rest of the ring
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     named_barrier(1, kConsumers);
-    // per-row largest magnitude, then convert in place to f16 * 2^e(m)
-    for (int mm = 0; mm < p.m; ++mm) {
-        float amax = 0.f;
-        for (int c = tid; c < per_row; c += kConsumers) {
-            const uint4 v = xsm[mm * xrow + c];
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                amax = fmaxf(amax, fabsf(bf2f(w4[i] & 0xFFFFu)));
-                amax = fmaxf(amax, fabsf(bf2f(w4[i] >> 16)));
+    {
+        // per-row largest magnitude, then conversion in place to f16 * 2^e(m): row r belongs
+        // to the kConsumerWarps / mp warps w with w / (kConsumerWarps / mp) == r (mp = M
+        // rounded up to a power of two), which share its amax through shared memory only
+        // when there is more than one of them
+        const int mp = p.m <= 1 ? 1 : (p.m <= 2 ? 2 : (p.m <= 4 ? 4 : 8));
+        const int wpr = kConsumerWarps / mp;
+        const int r = warp / wpr, part = warp - r * wpr;
+        uint32_t a = 0;
+        if (r < p.m)
+            for (int c = part * 32 + lane; c < per_row; c += wpr * 32) {
+                const uint4 v = xsm[r * xrow + c];
+                a = max(a, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                    __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
             }
-        }
+        a = max(a & 0xFFFFu, a >> 16);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-        if (lane == 0 && amax > 0.f) atomicMax(&s_amax[mm], __float_as_int(amax));
-    }
-    named_barrier(1, kConsumers);
-    for (int mm = 0; mm < p.m; ++mm) {
-        // amax in [2^E, 2^(E+1)) -> scale 2^(14-E) puts it in [2^14, 2^15), inside f16's range
-        const uint32_t bits = (uint32_t)s_amax[mm];
+        for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+        if (wpr > 1) {
+            if (lane == 0 && r < p.m) atomicMax(&s_amax[r], (int)a);
+            named_barrier(1, kConsumers);
+            a = r < p.m ? (uint32_t)s_amax[r] : 0u;
+        }
+        // a is the bf16 magnitude bit pattern of the row's largest |x| in the range; the scale
+        // 2^e puts that maximum in [2^14, 2^15), inside f16's range
         int e = 0;
-        const int E = (int)((bits >> 23) & 0xFF) - 127;
-        if (bits != 0 && E < 128) e = 14 - E;
+        if (a != 0u && a < 0x7F80u) e = 14 - ((int)(a >> 7) - 127);
         e = e > 126 ? 126 : (e < -126 ? -126 : e);
         const float sc = __uint_as_float((uint32_t)(e + 127) << 23);
-        if (tid == 0) s_descale[mm] = __uint_as_float((uint32_t)(127 - e) << 23);
-        for (int c = tid; c < per_row; c += kConsumers) {
-            uint4 v = xsm[mm * xrow + c];
-            uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        if (r < p.m) {
+            if (part == 0 && lane == 0) s_descale[r] = __uint_as_float((uint32_t)(127 - e) << 23);
+            for (int c = part * 32 + lane; c < per_row; c += wpr * 32) {
+                const uint4 v = xsm[r * xrow + c];
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                uint32_t h4[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const __half2 t = __floats2half2_rn(bf2f(w4[i] & 0xFFFFu) * sc, bf2f(w4[i] >> 16) * sc);
-                w4[i] = *reinterpret_cast<const uint32_t*>(&t);
+                for (int i = 0; i < 4; ++i) {
+                    const __half2 t = __floats2half2_rn(__uint_as_float(w4[i] << 16) * sc,
+                                                        __uint_as_float(w4[i] & 0xFFFF0000u) * sc);
+                    h4[i] = *reinterpret_cast<const uint32_t*>(&t);
+                }
+                xsm[r * xrow + c] = make_uint4(h4[0], h4[1], h4[2], h4[3]);
             }
-            xsm[mm * xrow + c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
     }
     named_barrier(1, kConsumers);
