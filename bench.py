@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import argparse
 import ctypes
+import hashlib
 import json
 import os
 import statistics
@@ -51,6 +52,39 @@ def parse():
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run this many eager steps and exit (for ncu launch lists)")
     return ap.parse_args()
+
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) that one ncu capture measured per
+# launch, for layer 0 of the sweep at M = 1 and M = 8 (profiles/nvfp4_gemv_sweep_dram_traffic.md).
+# They describe the kernel source with this SHA-256 only; for any other source the bench reports
+# traffic as null.
+TRAFFIC_SOURCE_SHA256 = "df7f0d3bf5ca319d28b7fdf2cf0de96fbbea481c13b04bac76891847cb3d1b4f"
+TRAFFIC_BYTES = {
+    ("L0.qkv", 1): 30119680, ("L0.o", 1): 18324480, ("L0.gate_up", 1): 107231232,
+    ("L0.down", 1): 50809344,
+    ("L0.qkv", 8): 29616896, ("L0.o", 8): 17837056, ("L0.gate_up", 8): 107827456,
+    ("L0.down", 8): 50468096,
+}
+KERNEL_SOURCE = os.path.join(ROOT, "nvfp4_weight_only_03_b200", "csrc", "nvfp4_gemv.cu")
+
+
+def measured_traffic(kind: str, bytes_of: dict, kind_of: dict):
+    """Mean ncu DRAM bytes per launch of `kind` over the captured launches, with the mean
+    algorithmic bytes of the same launches; None when the kernel source has changed since."""
+    try:
+        with open(KERNEL_SOURCE, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != TRAFFIC_SOURCE_SHA256:
+                return None
+    except OSError:
+        return None
+    keys = [k for k in TRAFFIC_BYTES if kind_of.get(k) == kind]
+    if not keys:
+        return None
+    meas = sum(TRAFFIC_BYTES[k] for k in keys) / len(keys)
+    alg = sum(bytes_of[k] for k in keys) / len(keys)
+    return {"bytes_per_launch": round(meas), "algorithmic_bytes_per_launch": round(alg),
+            "ratio": round(meas / alg, 4),
+            "launches": [f"{n}@M{m}" for (n, m) in keys]}
 
 
 def step_bytes(wl) -> dict:
@@ -136,9 +170,12 @@ def dist_setup(gpus: int):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:  # host-only runs (the rank logic's tests): gloo
+            dist.init_process_group("gloo", timeout=timeout)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -155,7 +192,8 @@ def max_over_ranks(v: float, world: int) -> float:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -354,10 +392,13 @@ def run_ours(args, world, rank, local):
     d = by_kind[dom]
     achieved = d["bytes"] / (d["us"] * 1e-6) / 1e9
     peak, peak_src = peaks()
-    traffic = None
+    kind_of = {key: kind for key, (kind, _) in per_launch.items()}
+    tr = measured_traffic(dom, bytes_of, kind_of)
+    traffic = tr["bytes_per_launch"] if tr else None
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
                 "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": peak_src,
+                "traffic_detail": tr,
                 "bytes_per_launch_avg": d["bytes"] / d["launches"],
                 "avg_launch_us": round(d["us"] / d["launches"], 3),
                 "timing": timing_src,
@@ -474,7 +515,7 @@ def run_reference(args, world, rank):
 
     for i in range(args.warmup):
         step(i)
-    steps = min(args.steps, 64)
+    steps = args.steps
     t0 = time.perf_counter()
     b = sum(step(i) for i in range(steps))
     dt = time.perf_counter() - t0
