@@ -263,8 +263,6 @@ __device__ __forceinline__ uint16_t f2bf(float v) {
     return (uint16_t)u;
 }
 
-__device__ __forceinline__ float bf2f(uint32_t b16) { return __uint_as_float(b16 << 16); }
-
 // A lane's decoded view of one stage for one stream: the multiply-ready k-step operands.
 __device__ __forceinline__ void compute_tile(float (&acc)[2][4], uint4 wa, uint4 wb, uint32_t sca,
                                              uint32_t scb, const uint4 (&xv)[4]) {
@@ -617,10 +615,9 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
                         }
                 }
                 named_barrier(1, kConsumers);
-                if (tid == 0) {
-                    __threadfence();
-                    st_release(p.flags + cta, 1u);
-                }
+                // the release store orders every consumer's partial stores (ordered before it by
+                // the barrier) ahead of the flag at GPU scope
+                if (tid == 0) st_release(p.flags + cta, 1u);
             } else {
                 if (cur_b + 1 != ku) {
                     // owner: the following CTAs hold the rest of this row group, each as the
