@@ -58,12 +58,12 @@ def parse():
 # launch, for layer 0 of the sweep at M = 1 and M = 8 (profiles/nvfp4_gemv_sweep_dram_traffic.md).
 # They describe the kernel source with this SHA-256 only; for any other source the bench reports
 # traffic as null.
-TRAFFIC_SOURCE_SHA256 = "df7f0d3bf5ca319d28b7fdf2cf0de96fbbea481c13b04bac76891847cb3d1b4f"
+TRAFFIC_SOURCE_SHA256 = "ca3f8ffccc982e68d1d5f2f10b8b2585767d99079cf776c3b6edcbbe8b2a9d0e"
 TRAFFIC_BYTES = {
-    ("L0.qkv", 1): 30119680, ("L0.o", 1): 18324480, ("L0.gate_up", 1): 107231232,
-    ("L0.down", 1): 50809344,
-    ("L0.qkv", 8): 29616896, ("L0.o", 8): 17837056, ("L0.gate_up", 8): 107827456,
-    ("L0.down", 8): 50468096,
+    ("L0.qkv", 1): 30119424, ("L0.o", 1): 18324736, ("L0.gate_up", 1): 106530816,
+    ("L0.down", 1): 50805760,
+    ("L0.qkv", 8): 29617408, ("L0.o", 8): 17837056, ("L0.gate_up", 8): 106519296,
+    ("L0.down", 8): 50459136,
 }
 KERNEL_SOURCE = os.path.join(ROOT, "nvfp4_weight_only_03_b200", "csrc", "nvfp4_gemv.cu")
 
