@@ -29,11 +29,13 @@
 //     instruction sequence serves every M, so row m of the output depends only on x row m:
 //     bitwise row invariance across M = 1..8.  Within a 16-row tile the mma's row r is weight
 //     row perm(r) (rows r and r+1 four apart), which makes the swizzled reads conflict-free.
-//   * x is staged once per CTA in shared memory as f16 (cp.async, then converted in place).
-//     Each x row m is scaled by a power of two 2^e(m) chosen from the row's largest magnitude
-//     in the CTA's k range (so it lands in [2^14, 2^15)); bf16 values convert exactly unless
-//     they are more than 2^31 times smaller than that maximum.  The partial sums are
-//     multiplied back by 2^-e(m) (exact) before they are combined.
+//   * x is staged once per CTA in shared memory as f16 (cp.async, then converted in place,
+//     each row by its own warps).  Each x row m is scaled by a power of two 2^e(m) chosen from
+//     the row's largest magnitude in the CTA's k range (so it lands in [2^14, 2^15)); bf16
+//     values convert exactly unless they are more than 2^31 times smaller than that maximum.
+//     The partial sums are multiplied back by 2^-e(m) (exact) before they are combined.  The
+//     producer issues at most kPrefetch units of weights before the consumers have requested
+//     x: a longer queue of weight boxes ahead of those requests would delay them.
 //   * Optional programmatic dependent launch: the weights stream in before the preceding
 //     kernel on the stream has finished; x, y and the workspace are touched only after
 //     griddepcontrol.wait.
