@@ -9,6 +9,11 @@ Metric: effective HBM GB/s = (packed weights + scales + bf16 activations + bf16 
 per step / device time per step.  Printed as one JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload sweep|attn_pairs]
+
+--workload attn_pairs measures nvfp4_gemv_multi instead: 8 layers x {k + v (2 x 1024x5120),
+q + gate (2 x 6144x5120)}, one launch per pair sharing x, M in {1, 8}; the same outputs as
+separate nvfp4_gemv launches are timed beside it.
 
 Under torchrun (N > 1) every rank runs an independent replica on its own GPU (the GEMV needs no
 collective); value = bytes of all ranks / max over ranks of the device time.
@@ -46,6 +51,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=("sweep", "attn_pairs"), default="sweep")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -573,6 +579,202 @@ def run_reference(args, world, rank):
                     "d2h_bytes_per_step": 0}}
 
 
+# ----------------------------------------------------------------------------------------------
+# several outputs sharing x (nvfp4_gemv_multi)
+
+PAIRS_LAYERS = 8
+PAIRS_ROWS = (1, 8)
+PAIRS_DESC = ("attention projection pairs sharing x: 8 layers x {k + v 2x1024x5120, q + gate "
+              "2x6144x5120} NVFP4, M in {1,8}, one nvfp4_gemv_multi launch per pair, back to back "
+              "on one stream")
+
+
+def run_pairs(args, world, rank, local):
+    import torch
+    import nvfp4_weight_only_03_b200 as nv
+    L = nv.lib()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    pairs = [synth.make("attn_kv"), synth.make("attn_qgate")]
+    # every layer streams its own copy of the pair weights (distinct device buffers: 330 MB per
+    # M pass, far above the 126 MB L2); x of each pair is the first projection's draw
+    layers = []
+    for _ in range(PAIRS_LAYERS):
+        for wl in pairs:
+            ws_ = [(torch.from_numpy(p.w.packed).to(dev), torch.from_numpy(p.w.scales).to(dev),
+                    p.w.g, p.n) for p in wl.projections]
+            x = torch.from_numpy(wl.projections[0].x.view(np.int16)).view(torch.bfloat16).to(dev)
+            ys = [torch.empty((8, n), dtype=torch.bfloat16, device=dev) for *_, n in ws_]
+            layers.append({"name": wl.name, "w": ws_, "x": x, "y": ys, "k": wl.projections[0].k})
+    ws = nv.workspace(dev)
+    flags = nv.FLAG_PREFETCH_WEIGHTS
+
+    def pass_bytes(m):
+        b = 0
+        for e in layers:
+            for (_, _, _, n) in e["w"]:
+                b += n * e["k"] // 2 + n * e["k"] // 16 + m * n * 2
+            b += m * e["k"] * 2
+        return b
+    step_bytes_ = sum(pass_bytes(m) for m in PAIRS_ROWS)
+
+    def calls(h, fused):
+        seq = []
+        for m in PAIRS_ROWS:
+            for e in layers:
+                if fused:
+                    outs = (nv.Output * len(e["w"]))()
+                    for o, ((W, S, g, n), y) in enumerate(zip(e["w"], e["y"])):
+                        outs[o].w, outs[o].s, outs[o].global_scale = W.data_ptr(), S.data_ptr(), g
+                        outs[o].y, outs[o].ldy, outs[o].n = y.data_ptr(), n, n
+                    seq.append((L.nvfp4_gemv_multi, (outs, len(e["w"]), e["x"].data_ptr(), e["k"],
+                                                    m, e["k"], ws.data_ptr(), ws.numel(), flags, h)))
+                else:
+                    for (W, S, g, n), y in zip(e["w"], e["y"]):
+                        seq.append((L.nvfp4_gemv_ex, (W.data_ptr(), S.data_ptr(), ctypes.c_float(g),
+                                                      e["x"].data_ptr(), e["k"], y.data_ptr(), n, m,
+                                                      n, e["k"], ws.data_ptr(), ws.numel(), flags,
+                                                      h)))
+        return seq
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def graph_of(fused):
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 3)):
+                for fn, a in calls(stream.cuda_stream, fused):
+                    if fn(*a) != 0:
+                        raise RuntimeError("launch failed")
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            seq = calls(torch.cuda.current_stream().cuda_stream, fused)
+            for fn, a in seq:
+                if fn(*a) != 0:
+                    raise RuntimeError("capture failed")
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        return g, len(seq)
+
+    def timed(g, steps):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            t0.record()
+            for _ in range(steps):
+                g.replay()
+            t1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(t0.elapsed_time(t1), world)
+
+    g_fused, n_fused = graph_of(True)
+    g_sep, n_sep = graph_of(False)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ms = timed(g_fused, args.steps)
+    clk = clocks.stop()
+    ms_sep = timed(g_sep, args.steps)
+    value = world * step_bytes_ * args.steps / (ms * 1e-3) / 1e9
+    value_sep = world * step_bytes_ * args.steps / (ms_sep * 1e-3) / 1e9
+    peak, peak_src = peaks()
+    per_launch_us = ms / args.steps * 1e3 / n_fused
+    bytes_avg = step_bytes_ / n_fused
+
+    # end to end through the public API: all x in from pinned host memory, all y back, per step
+    hx = torch.cat([e["x"].reshape(-1) for e in layers]).cpu().pin_memory()
+    dx = torch.empty_like(hx, device=dev)
+    xs, off = [], 0
+    for e in layers:
+        xs.append(dx[off:off + e["x"].numel()].view(8, e["k"]))
+        off += e["x"].numel()
+    ysz = sum(m * n for m in PAIRS_ROWS for e in layers for *_, n in e["w"])
+    hy = torch.empty(ysz, dtype=torch.bfloat16).pin_memory()
+    dy = torch.empty(ysz, dtype=torch.bfloat16, device=dev)
+    e2e_calls, off = [], 0
+    for m in PAIRS_ROWS:
+        for e, x in zip(layers, xs):
+            ys = []
+            for *_, n in e["w"]:
+                ys.append(dy[off:off + m * n].view(m, n))
+                off += m * n
+            e2e_calls.append(([(W, S, g) for W, S, g, _ in e["w"]], x[:m], ys))
+    cur = torch.cuda.current_stream()
+
+    def e2e_step():
+        dx.copy_(hx, non_blocking=True)
+        for wts, x, ys in e2e_calls:
+            nv.gemv_multi(wts, x, ys=ys, ws=ws, stream=cur, prefetch_weights=True)
+        hy.copy_(dy, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(cur)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    t1.record(cur)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(t0.elapsed_time(t1), world)
+    e2e = {"value": round(world * step_bytes_ * args.e2e_steps / (ms_e2e * 1e-3) / 1e9, 1),
+           "unit": "GB/s", "h2d_bytes_per_step": hx.numel() * 2, "d2h_bytes_per_step": ysz * 2,
+           "steps": args.e2e_steps, "api": "nvfp4_weight_only_03_b200.gemv_multi"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        threads = os.cpu_count() or 1
+        order = [(p, m) for m in PAIRS_ROWS for wl in pairs for p in wl.projections]
+        t_end = time.perf_counter() + args.cpu_seconds
+        b, n_calls, t_start = 0, 0, time.perf_counter()
+        while time.perf_counter() < t_end:
+            p, m = order[n_calls % len(order)]
+            x = pairs[0 if p.n == 1024 else 1].projections[0].x[:m]
+            oracle.gemv(p.w.packed, p.w.scales, p.w.g, x, rows=np.arange(256), threads=threads)
+            b += 256 * (p.k // 2 + p.k // 16) + m * p.k * 2 + m * 256 * 2
+            n_calls += 1
+        dt = time.perf_counter() - t_start
+        cpu = {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n_calls} calls of 256 output rows each, cycling over the four "
+                         f"projections and M in {{1,8}} ({dt:.1f} s)"}
+
+    del g_fused, g_sep
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4(e2m1+e4m3) x bf16 -> fp32 accumulate, bf16 out",
+            "data": "synthetic (seeded N(0,0.02) weights quantised to NVFP4, N(0,1) bf16 x)",
+            "config": {"workload": PAIRS_DESC, "rows": list(PAIRS_ROWS),
+                       "bytes_per_step": step_bytes_,
+                       "l2": "0.33 GB of weights per M pass > 126 MB L2; no flush",
+                       "launch": f"one CUDA graph per step ({n_fused} nvfp4_gemv_multi kernels, "
+                                 "programmatic dependent launch), persistent grid = SMs",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "kernel": "nvfp4_gemv_kernel<single, multi>",
+                         "achieved": round(bytes_avg / (per_launch_us * 1e-6) / 1e9, 1),
+                         "peak": peak, "unit": "GB/s",
+                         "frac": round(bytes_avg / (per_launch_us * 1e-6) / 1e9 / peak, 4),
+                         "traffic": None, "peak_source": peak_src,
+                         "bytes_per_launch_avg": bytes_avg,
+                         "avg_launch_us": round(per_launch_us, 3),
+                         "timing": "CUDA events around the K timed steps; every launch of the "
+                                   "step is this kernel"},
+            "separate_launches": {"value": round(value_sep, 1), "unit": "GB/s",
+                                  "launches_per_step": n_sep,
+                                  "ms_per_step": round(ms_sep / args.steps, 5),
+                                  "what": "the same outputs as one nvfp4_gemv launch each"},
+            "e2e": e2e, "gpu_launches": n_fused * args.steps, "clocks": clk}
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    return line
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -583,7 +785,7 @@ def main():
             print(json.dumps(line), flush=True)
         return
     world, rank, local = dist_setup(args.gpus)
-    line = run_ours(args, world, rank, local)
+    line = (run_pairs if args.workload == "attn_pairs" else run_ours)(args, world, rank, local)
     if line is not None and rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -68,6 +68,7 @@ typedef enum {
 } nvfp4_status;
 
 #define NVFP4_MAX_ROWS 8
+#define NVFP4_MAX_OUTPUTS 4
 #define NVFP4_GROUP 16
 #define NVFP4_LAYOUT_VERSION 1
 
@@ -132,6 +133,38 @@ int nvfp4_gemv_dual_ex(const uint8_t* w_gate, const uint8_t* s_gate, float globa
                        int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
                        void* workspace, size_t workspace_bytes, uint32_t flags,
                        cudaStream_t stream);
+
+/* One output of nvfp4_gemv_multi: an N x K weight in the format above, its global scale, and
+ * where its N outputs go.  w: 16-byte aligned; s, y: 2-byte aligned; ldy >= n. */
+typedef struct {
+    const uint8_t* w;      /* packed weights [n][K/2] */
+    const uint8_t* s;      /* scale codes [n][K/16] */
+    float global_scale;
+    void* y;               /* bf16 [M][ldy] */
+    int64_t ldy;
+    int64_t n;             /* rows of this weight; 0 skips the output */
+} nvfp4_output_t;
+
+/* Several single-output GEMVs that share x and K, in one pass: for every output o,
+ *   y_o[m][n] = bf16_rn( g_o * sum_k E2M1(W_o[n][k]) * E4M3(S_o[n][k/16]) * x[m][k] ).
+ * The decode plan runs such groups as one launch: the attention k and v projections (the GB10
+ * plan's two-output "w4a16_gemv_dual", 16 launches per step) and the gated attention's q and gate
+ * ("w4a16_gemv_qg") ("Blueprint - circuit executor" page, table "Kernels the plan launches").
+ *   outputs: `count` (1..NVFP4_MAX_OUTPUTS) descriptors, host memory, read during the call only.
+ *   x, ldx, m, k, workspace, flags, stream: as nvfp4_gemv_ex.
+ * The row groups of all outputs form one stream-K split over the GPU, so one launch streams
+ * every weight.  When K is so large that nvfp4_gemv itself would split an output's rows over
+ * several launches, and the outputs together exceed one launch, each output runs as its own
+ * nvfp4_gemv_ex call instead.  Either way each result depends only on (every output's n, K,
+ * SM count) and x's row: row invariance over M = 1..8 and determinism hold as for nvfp4_gemv,
+ * and the result of an output alone (count 1) is bitwise that of nvfp4_gemv_ex.  Output
+ * buffers must not overlap one another, x or the weights.
+ * Errors: NVFP4_ERR_NULL (outputs NULL, or as nvfp4_gemv for an output), NVFP4_ERR_SHAPE
+ * (count out of range, or as nvfp4_gemv), and those of nvfp4_gemv_ex, checked output by output
+ * before anything is enqueued. */
+int nvfp4_gemv_multi(const nvfp4_output_t* outputs, int count, const void* x, int64_t ldx,
+                     int m, int64_t k, void* workspace, size_t workspace_bytes, uint32_t flags,
+                     cudaStream_t stream);
 
 /* nvfp4_gemv for a caller that cannot provide a workspace.  The NVFP4 pages describe no such
  * call: it is a library convenience.  It serves callers that may not allocate device memory

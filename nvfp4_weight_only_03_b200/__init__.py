@@ -7,6 +7,7 @@ missing or the device is not a B200 the calls raise.
 
     y = gemv(w, s, g, x)                      # y[m][n] = bf16(g * sum_k e2m1(w) e4m3(s) x)
     o = gemv_dual(wg, sg, gg, wu, su, gu, x)  # o = bf16(silu(gate) * up)
+    k_, v_ = gemv_multi([(wk, sk, gk), (wv, sv, gv)], x)  # several outputs sharing x, one pass
 
 w: uint8 [N][K/2] packed e2m1 (low nibble = even k), s: uint8 [N][K/16] e4m3 scale codes,
 g: float global scale, x: bfloat16 [M][K] (M = 1..8, row stride may exceed K).
@@ -27,6 +28,7 @@ STATUS = {0: "NVFP4_OK", -1: "NVFP4_ERR_NULL", -2: "NVFP4_ERR_SHAPE", -3: "NVFP4
           -4: "NVFP4_ERR_ALIGN", -5: "NVFP4_ERR_ARCH", -6: "NVFP4_ERR_LAUNCH",
           -7: "NVFP4_ERR_WORKSPACE"}
 MAX_ROWS = 8
+MAX_OUTPUTS = 4
 GROUP = 16
 FLAG_PREFETCH_WEIGHTS = 1
 
@@ -35,6 +37,12 @@ class Nvfp4Error(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class Output(ctypes.Structure):
+    """nvfp4_output_t: one output of nvfp4_gemv_multi."""
+    _fields_ = [("w", ctypes.c_void_p), ("s", ctypes.c_void_p), ("global_scale", ctypes.c_float),
+                ("y", ctypes.c_void_p), ("ldy", ctypes.c_int64), ("n", ctypes.c_int64)]
 
 
 class PackInfo(ctypes.Structure):
@@ -70,12 +78,14 @@ def lib():
                                          vp, i64, c_int, i64, i64, vp, sz, ctypes.c_uint32, vp]
         L.nvfp4_gemv_noalloc.argtypes = [vp, vp, ctypes.c_float, vp, i64, vp, i64, c_int, i64,
                                          i64, vp]
+        L.nvfp4_gemv_multi.argtypes = [ctypes.POINTER(Output), c_int, vp, i64, c_int, i64, vp,
+                                       sz, ctypes.c_uint32, vp]
         L.nvfp4_workspace_error.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
         L.nvfp4_status_string.argtypes = [c_int]
         L.nvfp4_status_string.restype = ctypes.c_char_p
         for f in (L.nvfp4_pack_info, L.nvfp4_workspace_bytes, L.nvfp4_gemv, L.nvfp4_gemv_dual,
                   L.nvfp4_gemv_ex, L.nvfp4_gemv_dual_ex, L.nvfp4_gemv_noalloc,
-                  L.nvfp4_workspace_error):
+                  L.nvfp4_gemv_multi, L.nvfp4_workspace_error):
             f.restype = c_int
         _lib = L
     return _lib
@@ -205,3 +215,34 @@ def gemv_dual(wg: torch.Tensor, sg: torch.Tensor, gg: float, wu: torch.Tensor, s
                                   m, n, k, ws.data_ptr(), ws.numel(), flags, _stream(stream))
     _check(st, "nvfp4_gemv_dual")
     return y
+
+
+def gemv_multi(weights, x: torch.Tensor, ys=None, ws: torch.Tensor = None, stream=None,
+               prefetch_weights: bool = False) -> list:
+    """Several GEMVs sharing x in one pass (nvfp4_gemv_multi): weights is a list of up to
+    MAX_OUTPUTS (w, s, g) triples with the same K; returns [y_0, y_1, ...], y_o the GEMV of
+    weight o as gemv computes it.  ys: optional preallocated outputs, one per weight."""
+    weights = list(weights)
+    if not 1 <= len(weights) <= MAX_OUTPUTS:
+        raise ValueError(f"1..{MAX_OUTPUTS} weights, got {len(weights)}")
+    shapes = [_weight_args(w, s) for w, s, _ in weights]
+    k = shapes[0][1]
+    if any(kk != k for _, kk in shapes):
+        raise ValueError("all weights must have the same K")
+    x, m, ldx = _x_args(x, k)
+    ys = [None] * len(weights) if ys is None else list(ys)
+    if len(ys) != len(weights):
+        raise ValueError("one output per weight")
+    outs = (Output * len(weights))()
+    result = []
+    for o, ((w, s, g), (n, _), y) in enumerate(zip(weights, shapes, ys)):
+        y, ldy = _out(y, m, n, x)
+        result.append(y)
+        outs[o].w, outs[o].s, outs[o].global_scale = w.data_ptr(), s.data_ptr(), float(g)
+        outs[o].y, outs[o].ldy, outs[o].n = y.data_ptr(), ldy, n
+    ws = workspace(x.device) if ws is None else ws
+    flags = FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0
+    st = lib().nvfp4_gemv_multi(outs, len(weights), x.data_ptr(), ldx, m, k, ws.data_ptr(),
+                                ws.numel(), flags, _stream(stream))
+    _check(st, "nvfp4_gemv_multi")
+    return result

@@ -114,15 +114,22 @@ template <bool DUAL> using Cfg = typename CfgSel<DUAL>::type;
 
 enum ScaleMode { kScaleTma = 0, kScaleAsync8 = 1, kScaleScalar = 2 };
 
+// Outputs of one launch of the single-stream kernel: several weight matrices with the same K
+// share x, their row groups concatenated in output order (one output for nvfp4_gemv).  The dual
+// kernel has one output fed by two weight streams (index = stream).
+constexpr int kMaxOutputs = NVFP4_MAX_OUTPUTS;
+
 struct Params {
-    const uint8_t* s[2];
-    float g[2];          // global scales
+    const uint8_t* s[kMaxOutputs];  // scale codes, per output (dual: per stream)
+    float g[kMaxOutputs];           // global scales, per output (dual: per stream)
+    uint16_t* y[kMaxOutputs];       // outputs (dual: y[0])
+    int64_t ldy[kMaxOutputs];
+    int64_t n[kMaxOutputs];         // rows of each output (dual: n[0])
+    int64_t gend[kMaxOutputs];      // row groups of outputs 0..o together
+    int outs;                       // outputs (1 for the dual)
     const uint16_t* x;
     int64_t ldx;
-    uint16_t* y;
-    int64_t ldy;
     int m;
-    int64_t n;
     int64_t k;
     int ku;              // 256-k units along K (the last may be partial)
     int64_t units;       // row groups * ku
@@ -132,6 +139,15 @@ struct Params {
     float* partial;      // [grid][2][kPartialFloats]
     uint32_t* flags;     // [grid]
     int32_t* error;
+};
+
+// Tensor maps of one launch: packed weights and scale codes per output (dual: per stream).
+// A kernel instance carries only as many as it can use.
+template <bool DUAL, bool MULTI>
+struct Maps {
+    static constexpr int kCount = DUAL ? 2 : (MULTI ? kMaxOutputs : 1);
+    CUtensorMap w[kCount];
+    CUtensorMap s[kCount];
 };
 
 // ------------------------------------------------------------------------------------------
@@ -305,30 +321,37 @@ __device__ __forceinline__ int perm_row(int r) { return (r & 8) | ((r >> 1) & 3)
 // Byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled box of 128-byte rows.
 __device__ __forceinline__ int swz(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
-// Write this lane's outputs of one tile: c0 (row ra, col 2q), c1 (ra, 2q+1), c2 (rb, 2q),
-// c3 (rb, 2q+1).
-__device__ __forceinline__ void store_tile(const Params& p, int64_t ra, int64_t rb, int q,
+// Write this lane's outputs of one tile of output o (rows ra, rb local to it): c0 (row ra,
+// col 2q), c1 (ra, 2q+1), c2 (rb, 2q), c3 (rb, 2q+1).
+__device__ __forceinline__ void store_tile(const Params& p, int o, int64_t ra, int64_t rb, int q,
                                            const float (&v)[4]) {
     const int c0 = 2 * q, c1 = 2 * q + 1;
+    uint16_t* const y = p.y[o];
+    const int64_t ldy = p.ldy[o], n = p.n[o];
     if (c0 < p.m) {
-        if (ra < p.n) p.y[c0 * p.ldy + ra] = f2bf(v[0]);
-        if (rb < p.n) p.y[c0 * p.ldy + rb] = f2bf(v[2]);
+        if (ra < n) y[c0 * ldy + ra] = f2bf(v[0]);
+        if (rb < n) y[c0 * ldy + rb] = f2bf(v[2]);
     }
     if (c1 < p.m) {
-        if (ra < p.n) p.y[c1 * p.ldy + ra] = f2bf(v[1]);
-        if (rb < p.n) p.y[c1 * p.ldy + rb] = f2bf(v[3]);
+        if (ra < n) y[c1 * ldy + ra] = f2bf(v[1]);
+        if (rb < n) y[c1 * ldy + rb] = f2bf(v[3]);
     }
+}
+
+// Output holding global row group rg (the groups of outputs 0..o end at p.gend[o]).
+__device__ __forceinline__ int output_of(const Params& p, int64_t rg) {
+    int o = 0;
+    while (o + 1 < p.outs && rg >= p.gend[o]) ++o;
+    return o;
 }
 
 // ------------------------------------------------------------------------------------------
 // the kernel
 
-template <bool DUAL>
+// MULTI: the single-stream kernel over several outputs (nvfp4_gemv_multi); otherwise one output.
+template <bool DUAL, bool MULTI>
 __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
-    nvfp4_gemv_kernel(const Params p, const __grid_constant__ CUtensorMap tw0,
-                      const __grid_constant__ CUtensorMap tw1,
-                      const __grid_constant__ CUtensorMap ts0,
-                      const __grid_constant__ CUtensorMap ts1) {
+    nvfp4_gemv_kernel(const Params p, const __grid_constant__ Maps<DUAL, MULTI> maps) {
     using C = Cfg<DUAL>;
     constexpr int NS = C::kStreams;
     const int S = p.stages;
@@ -383,6 +406,10 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
         const int64_t srow = p.k >> 4;
         int64_t rg = rg0;
         int b = b0;
+        // output of row group rg and its first row group (the single kernel's outputs follow
+        // one another; the dual's two streams share one output)
+        int o = MULTI ? output_of(p, rg0) : 0;
+        int64_t gbase = o > 0 ? p.gend[o - 1] : 0;
         bool ok = true;
         int slot = 0;
         uint32_t phase = 0;  // parity of the ring pass in progress
@@ -407,14 +434,16 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
             }
             uint8_t* dst = ring + slot * C::kStageBytes;
             uint8_t* sdst = dst + NS * kWBytes;
-            const int y = (int)(rg * kRows);
+            const int y = (int)((rg - gbase) * kRows);  // first row of the unit in output o
             if (lane == 0) {
                 mbar_expect_tx(&full_bar[slot], tx);
-                tma_load_2d(dst, &tw0, b * kWRowBytes, y, &full_bar[slot]);
-                if (DUAL) tma_load_2d(dst + kWBytes, &tw1, b * kWRowBytes, y, &full_bar[slot]);
+                tma_load_2d(dst, &maps.w[o], b * kWRowBytes, y, &full_bar[slot]);
+                if constexpr (DUAL)
+                    tma_load_2d(dst + kWBytes, &maps.w[1], b * kWRowBytes, y, &full_bar[slot]);
                 if (mode == kScaleTma) {
-                    tma_load_2d(sdst, &ts0, b * kSRowBytes, y, &full_bar[slot]);
-                    if (DUAL) tma_load_2d(sdst + kSBytes, &ts1, b * kSRowBytes, y, &full_bar[slot]);
+                    tma_load_2d(sdst, &maps.s[o], b * kSRowBytes, y, &full_bar[slot]);
+                    if constexpr (DUAL)
+                        tma_load_2d(sdst + kSBytes, &maps.s[1], b * kSRowBytes, y, &full_bar[slot]);
                 }
             }
             if (mode != kScaleTma) {
@@ -423,8 +452,8 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
                 for (int s = 0; s < NS; ++s)
                     for (int r = lane; r < kRows; r += 32) {
                         const int64_t row = (int64_t)y + r;
-                        const bool vrow = row < p.n;
-                        const uint8_t* src = p.s[s] + (vrow ? row * srow : 0);
+                        const bool vrow = row < p.n[o];
+                        const uint8_t* src = p.s[o + s] + (vrow ? row * srow : 0);
                         uint8_t* d = sdst + s * kSBytes + r * kSRowBytes;
                         const int64_t g0 = (int64_t)b * kSRowBytes;
                         if (mode == kScaleAsync8) {
@@ -446,6 +475,7 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
             if (++b == ku) {
                 b = 0;
                 ++rg;
+                if (MULTI && o + 1 < p.outs && rg == p.gend[o]) gbase = p.gend[o++];
             }
             if (++slot == S) {
                 slot = 0;
@@ -655,9 +685,11 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
                     named_barrier(1, kConsumers);
                     for (int c = tid; c < nc; c += kConsumers) p.flags[cta + 1 + c] = 0u;
                 }
+                const int o = MULTI ? output_of(p, cur_rg) : 0;
+                const int64_t grow = (cur_rg - (o > 0 ? p.gend[o - 1] : 0)) * kRows;
 #pragma unroll
                 for (int t = 0; t < kTiles; ++t) {
-                    const int64_t row0 = cur_rg * kRows + (warp * kTiles + t) * 16;
+                    const int64_t row0 = grow + (warp * kTiles + t) * 16;
                     float v[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -666,10 +698,10 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
                             const float b = tot[1][t][e] * p.g[1];
                             v[e] = a / (1.0f + expf(-a)) * b;
                         } else {
-                            v[e] = tot[0][t][e] * p.g[0];
+                            v[e] = tot[0][t][e] * p.g[o];
                         }
                     }
-                    store_tile(p, row0 + pr_a, row0 + pr_b, q, v);
+                    store_tile(p, o, row0 + pr_a, row0 + pr_b, q, v);
                 }
             }
             seg_b0 = 0;
@@ -693,7 +725,7 @@ struct DeviceInfo {
     int sms = 0;
 };
 DeviceInfo g_dev[64];
-bool g_attr_set[2][64];
+bool g_attr_set[3][64];  // single, dual, multi
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -787,11 +819,43 @@ bool encode_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t col
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// One output of a launch: its weight streams (two for the dual, gate then up), their global
+// scales, and its rows.
+struct Span {
+    const uint8_t* w[2];
+    const uint8_t* s[2];
+    float g[2];
+    void* y;
+    int64_t ldy;
+    int64_t n;
+};
+
+constexpr size_t kXSlotBytes = (size_t)2 * kSlotU4 * 16;  // staged x per unit per row: 512 B
+
+// Row groups one launch may hold for this K, or -1 for no limit: the staged x of a CTA's range
+// (M rows x the range's 256-k units, sized for M = 8 so that the split never depends on M) must
+// fit shared memory beside the smallest ring.
 template <bool DUAL>
-int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, const void* x,
-           int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws,
-           size_t ws_bytes, uint32_t flags, cudaStream_t stream) {
+int64_t max_groups_per_launch(int64_t k, int sms) {
     using C = Cfg<DUAL>;
+    const int ku = (int)((k + kUnitK - 1) / kUnitK);
+    const size_t mx = NVFP4_MAX_ROWS;
+    const int64_t max_slots = (int64_t)((kSmemMax - 1024 - kMinStages * C::kStageBytes -
+                                         mx * kRowPadU4 * 16) /
+                                        (mx * kXSlotBytes));
+    if (max_slots >= ku) return -1;
+    const int64_t groups = (int64_t)sms * max_slots / ku;
+    return groups > 0 ? groups : 1;
+}
+
+// One launch over the spans' row groups, concatenated in order (the dual takes one span; more
+// than one span needs MULTI).
+template <bool DUAL, bool MULTI>
+int launch_spans(const Span* sp, int count, const void* x, int64_t ldx, int m, int64_t k,
+                 void* ws, size_t ws_bytes, uint32_t flags, cudaStream_t stream) {
+    using C = Cfg<DUAL>;
+    static_assert(!(DUAL && MULTI), "the dual kernel has one output");
+    if (count > Maps<DUAL, MULTI>::kCount / (DUAL ? 2 : 1)) return NVFP4_ERR_SHAPE;
     constexpr int NS = C::kStreams;
     int dev = 0;
     DeviceInfo* di = nullptr;
@@ -802,119 +866,135 @@ int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, co
     if (ws_bytes < need) return NVFP4_ERR_WORKSPACE;
 
     if (k == 0) {  // empty sum: y = 0 (silu(0) * 0 = 0 for the dual)
-        if (cudaMemset2DAsync(y, (size_t)ldy * 2, 0, (size_t)n * 2, (size_t)m, stream) !=
-            cudaSuccess) {
-            cudaGetLastError();
-            return NVFP4_ERR_LAUNCH;
-        }
+        for (int o = 0; o < count; ++o)
+            if (cudaMemset2DAsync(sp[o].y, (size_t)sp[o].ldy * 2, 0, (size_t)sp[o].n * 2,
+                                  (size_t)m, stream) != cudaSuccess) {
+                cudaGetLastError();
+                return NVFP4_ERR_LAUNCH;
+            }
         return NVFP4_OK;
     }
 
-    if (!g_attr_set[DUAL][dev]) {
-        if (cudaFuncSetAttribute(nvfp4_gemv_kernel<DUAL>,
+    const int variant = DUAL ? 1 : (MULTI ? 2 : 0);
+    if (!g_attr_set[variant][dev]) {
+        if (cudaFuncSetAttribute(nvfp4_gemv_kernel<DUAL, MULTI>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) !=
             cudaSuccess) {
             cudaGetLastError();
             return NVFP4_ERR_LAUNCH;
         }
-        g_attr_set[DUAL][dev] = true;
+        g_attr_set[variant][dev] = true;
     }
 
     // how the producer moves the scale codes: TMA needs 16-byte aligned scale rows
     int scale_mode = kScaleTma;
-    for (int i = 0; i < NS; ++i) {
-        if ((k % kUnitK) != 0 || misaligned(s[i], 16)) scale_mode = kScaleAsync8;
-    }
-    if (scale_mode == kScaleAsync8) {
+    for (int o = 0; o < count; ++o)
         for (int i = 0; i < NS; ++i)
-            if ((k % kBlockK) != 0 || misaligned(s[i], 8)) scale_mode = kScaleScalar;
+            if ((k % kUnitK) != 0 || misaligned(sp[o].s[i], 16)) scale_mode = kScaleAsync8;
+    if (scale_mode == kScaleAsync8) {
+        for (int o = 0; o < count; ++o)
+            for (int i = 0; i < NS; ++i)
+                if ((k % kBlockK) != 0 || misaligned(sp[o].s[i], 8)) scale_mode = kScaleScalar;
     }
 
     const int ku = (int)((k + kUnitK - 1) / kUnitK);
-    const size_t slot_bytes = (size_t)2 * kSlotU4 * 16;  // 512 B of staged x per unit per row
-    const int max_grid = di->sms;
-    // Rows per launch: the ring plus the staged x (M rows x units of a CTA's range) must fit
-    // shared memory; a range spans at most ceil(units / grid) units, capped at ku.  Sized for
-    // the largest M so that the work split never depends on M.
-    int64_t rows_per_launch = n;
-    {
-        const size_t mx = NVFP4_MAX_ROWS;
-        const int64_t max_slots = (int64_t)((kSmemMax - 1024 - kMinStages * C::kStageBytes -
-                                             mx * kRowPadU4 * 16) /
-                                            (mx * slot_bytes));
-        if (max_slots < ku) {
-            const int64_t groups = (int64_t)max_grid * max_slots / ku;
-            const int64_t cap = (groups > 0 ? groups : 1) * C::kRows;
-            if (cap < rows_per_launch) rows_per_launch = cap;
+    Params p;
+    memset(&p, 0, sizeof(p));
+    Maps<DUAL, MULTI> maps;
+    memset(&maps, 0, sizeof(maps));
+    int64_t groups = 0;
+    for (int o = 0; o < count; ++o) {
+        const Span& a = sp[o];
+        // map / pointer slot of output o (single) or of stream i (dual)
+        for (int i = 0; i < NS; ++i) {
+            const int slot = DUAL ? i : o;
+            p.s[slot] = a.s[i];
+            p.g[slot] = a.g[i];
+            if (!encode_map(&maps.w[slot], a.w[i], a.n, k / 2, kWRowBytes, C::kRows,
+                            CU_TENSOR_MAP_SWIZZLE_128B))
+                return NVFP4_ERR_LAUNCH;
+            if (scale_mode == kScaleTma &&
+                !encode_map(&maps.s[slot], a.s[i], a.n, k / 16, kSRowBytes, C::kRows,
+                            CU_TENSOR_MAP_SWIZZLE_NONE))
+                return NVFP4_ERR_LAUNCH;
         }
+        p.y[o] = static_cast<uint16_t*>(a.y);
+        p.ldy[o] = a.ldy;
+        p.n[o] = a.n;
+        groups += (a.n + C::kRows - 1) / C::kRows;
+        p.gend[o] = groups;
     }
-
+    p.outs = count;
+    p.x = static_cast<const uint16_t*>(x);
+    p.ldx = ldx;
+    p.m = m;
+    p.k = k;
+    p.ku = ku;
+    p.units = groups * ku;
+    const int max_grid = di->sms;
+    p.grid = (int)(p.units < max_grid ? p.units : max_grid);
+    p.scale_mode = scale_mode;
     char* wsb = static_cast<char*>(ws);
-    for (int64_t r0 = 0; r0 < n; r0 += rows_per_launch) {
-        const int64_t nn = (n - r0) < rows_per_launch ? (n - r0) : rows_per_launch;
-        Params p;
-        CUtensorMap tw[2], tsc[2];
-        memset(tw, 0, sizeof(tw));
-        memset(tsc, 0, sizeof(tsc));
-        for (int i = 0; i < 2; ++i) {
-            const int src = DUAL ? i : 0;
-            p.s[i] = s[src] + r0 * (k / 16);
-            p.g[i] = gs[src];
-            if (i == 0 || DUAL) {
-                if (!encode_map(&tw[i], w[src] + r0 * (k / 2), nn, k / 2, kWRowBytes, C::kRows,
-                                CU_TENSOR_MAP_SWIZZLE_128B))
-                    return NVFP4_ERR_LAUNCH;
-                if (scale_mode == kScaleTma &&
-                    !encode_map(&tsc[i], s[src] + r0 * (k / 16), nn, k / 16, kSRowBytes, C::kRows,
-                                CU_TENSOR_MAP_SWIZZLE_NONE))
-                    return NVFP4_ERR_LAUNCH;
-            }
-        }
-        if (!DUAL) {
-            tw[1] = tw[0];
-            tsc[1] = tsc[0];
-        }
-        p.x = static_cast<const uint16_t*>(x);
-        p.ldx = ldx;
-        p.y = static_cast<uint16_t*>(y) + r0;
-        p.ldy = ldy;
-        p.m = m;
-        p.n = nn;
-        p.k = k;
-        p.ku = ku;
-        p.units = ((nn + C::kRows - 1) / C::kRows) * ku;
-        p.grid = (int)(p.units < max_grid ? p.units : max_grid);
-        p.scale_mode = scale_mode;
-        p.partial = reinterpret_cast<float*>(wsb + partial_off);
-        p.flags = reinterpret_cast<uint32_t*>(wsb + flags_off);
-        p.error = reinterpret_cast<int32_t*>(wsb);
-        const int64_t max_range = (p.units + p.grid - 1) / p.grid;
-        const int slots = (int)(max_range < ku ? max_range : ku);
-        const size_t xbytes = (size_t)m * ((size_t)slots * slot_bytes + kRowPadU4 * 16);
-        int stages = (int)((kSmemMax - 1024 - xbytes) / C::kStageBytes);
-        stages = stages > kMaxStages ? kMaxStages : stages;
-        if (stages < kMinStages) return NVFP4_ERR_LAUNCH;  // cannot happen: the split bounds x
-        p.stages = stages;
-        const size_t smem = 1024 + (size_t)stages * C::kStageBytes + xbytes;
+    p.partial = reinterpret_cast<float*>(wsb + partial_off);
+    p.flags = reinterpret_cast<uint32_t*>(wsb + flags_off);
+    p.error = reinterpret_cast<int32_t*>(wsb);
+    const int64_t max_range = (p.units + p.grid - 1) / p.grid;
+    const int slots = (int)(max_range < ku ? max_range : ku);
+    const size_t xbytes = (size_t)m * ((size_t)slots * kXSlotBytes + kRowPadU4 * 16);
+    int stages = (int)((kSmemMax - 1024 - xbytes) / C::kStageBytes);
+    stages = stages > kMaxStages ? kMaxStages : stages;
+    if (stages < kMinStages) return NVFP4_ERR_LAUNCH;  // cannot happen: the split bounds x
+    p.stages = stages;
+    const size_t smem = 1024 + (size_t)stages * C::kStageBytes + xbytes;
 
-        cudaLaunchConfig_t cfg;
-        memset(&cfg, 0, sizeof(cfg));
-        cfg.gridDim = dim3(p.grid);
-        cfg.blockDim = dim3(C::kThreads);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        if (flags & NVFP4_FLAG_PREFETCH_WEIGHTS) {
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(p.grid);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    if (flags & NVFP4_FLAG_PREFETCH_WEIGHTS) {
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    if (cudaLaunchKernelEx(&cfg, nvfp4_gemv_kernel<DUAL, MULTI>, p, maps) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_LAUNCH;
+    }
+    return NVFP4_OK;
+}
+
+// One output (one or two weight streams), split into launches of at most
+// max_groups_per_launch row groups.
+template <bool DUAL>
+int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, const void* x,
+           int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws,
+           size_t ws_bytes, uint32_t flags, cudaStream_t stream) {
+    using C = Cfg<DUAL>;
+    constexpr int NS = C::kStreams;
+    int dev = 0;
+    DeviceInfo* di = nullptr;
+    int st = device_info(&dev, &di);
+    if (st != NVFP4_OK) return st;
+    const int64_t cap = max_groups_per_launch<DUAL>(k, di->sms);
+    const int64_t rows_per_launch = cap < 0 ? n : cap * C::kRows;
+    for (int64_t r0 = 0; r0 < n; r0 += rows_per_launch) {
+        Span a;
+        memset(&a, 0, sizeof(a));
+        for (int i = 0; i < NS; ++i) {
+            a.w[i] = w[i] + r0 * (k / 2);
+            a.s[i] = s[i] + r0 * (k / 16);
+            a.g[i] = gs[i];
         }
-        if (cudaLaunchKernelEx(&cfg, nvfp4_gemv_kernel<DUAL>, p, tw[0], tw[1], tsc[0], tsc[1]) !=
-            cudaSuccess) {
-            cudaGetLastError();
-            return NVFP4_ERR_LAUNCH;
-        }
+        a.y = static_cast<uint16_t*>(y) + r0;
+        a.ldy = ldy;
+        a.n = (n - r0) < rows_per_launch ? (n - r0) : rows_per_launch;
+        if ((st = launch_spans<DUAL, false>(&a, 1, x, ldx, m, k, ws, ws_bytes, flags, stream)) !=
+            NVFP4_OK)
+            return st;
     }
     return NVFP4_OK;
 }
@@ -1052,6 +1132,56 @@ int nvfp4_gemv_dual(const uint8_t* w_gate, const uint8_t* s_gate, float global_g
                     void* workspace, size_t workspace_bytes, cudaStream_t stream) {
     return nvfp4_gemv_dual_ex(w_gate, s_gate, global_gate, w_up, s_up, global_up, x, ldx, y, ldy,
                               m, n, k, workspace, workspace_bytes, 0u, stream);
+}
+
+int nvfp4_gemv_multi(const nvfp4_output_t* outputs, int count, const void* x, int64_t ldx,
+                     int m, int64_t k, void* workspace, size_t workspace_bytes, uint32_t flags,
+                     cudaStream_t stream) {
+    if (!outputs) return NVFP4_ERR_NULL;
+    if (count < 1 || count > NVFP4_MAX_OUTPUTS) return NVFP4_ERR_SHAPE;
+    Span sp[kMaxOutputs];
+    int used = 0;
+    for (int o = 0; o < count; ++o) {
+        const nvfp4_output_t& a = outputs[o];
+        bool noop = false;
+        int st = check_common(x, ldx, a.y, a.ldy, m, a.n, k, workspace, flags, &noop);
+        if (st != NVFP4_OK) return st;
+        if (noop) continue;  // M == 0 or no rows: nothing to write
+        if (k > 0 && (st = check_weight(a.w, a.s)) != NVFP4_OK) return st;
+        Span& b = sp[used++];
+        memset(&b, 0, sizeof(b));
+        b.w[0] = a.w;
+        b.s[0] = a.s;
+        b.g[0] = a.global_scale;
+        b.y = a.y;
+        b.ldy = a.ldy;
+        b.n = a.n;
+    }
+    if (used == 0) return NVFP4_OK;
+    int dev = 0;
+    DeviceInfo* di = nullptr;
+    int st = device_info(&dev, &di);
+    if (st != NVFP4_OK) return st;
+    using C = Cfg<false>;
+    int64_t groups = 0;
+    for (int o = 0; o < used; ++o) groups += (sp[o].n + C::kRows - 1) / C::kRows;
+    const int64_t cap = max_groups_per_launch<false>(k, di->sms);
+    if (used == 1)  // the one-output kernel: bitwise nvfp4_gemv_ex, which also splits its rows
+        return launch<false>(sp[0].w, sp[0].s, sp[0].g, x, ldx, sp[0].y, sp[0].ldy, m, sp[0].n,
+                             k, workspace, workspace_bytes, flags, stream);
+    if (cap < 0 || groups <= cap)
+        return launch_spans<false, true>(sp, used, x, ldx, m, k, workspace, workspace_bytes,
+                                         flags, stream);
+    // too many row groups for one launch at this K: each output as nvfp4_gemv runs it
+    for (int o = 0; o < used; ++o) {
+        const uint8_t* w_[1] = {sp[o].w[0]};
+        const uint8_t* s_[1] = {sp[o].s[0]};
+        const float g_[1] = {sp[o].g[0]};
+        if ((st = launch<false>(w_, s_, g_, x, ldx, sp[o].y, sp[o].ldy, m, sp[o].n, k, workspace,
+                                workspace_bytes, flags, stream)) != NVFP4_OK)
+            return st;
+    }
+    return NVFP4_OK;
 }
 
 int nvfp4_workspace_error(const void* workspace, size_t workspace_bytes, cudaStream_t stream,

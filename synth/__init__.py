@@ -193,6 +193,11 @@ _RECIPES = {
     "sweep": ([(f"L{l}.{nm}", n, k, d) for l in range(4) for (nm, n, k, d) in
                (("qkv", 10240, 5120, False), ("o", 5120, 6144, False),
                 ("gate_up", 17408, 5120, True), ("down", 5120, 17408, False))], 4, (1, 2, 4, 8)),
+    # several weights sharing one x (nvfp4_gemv_multi): the gated attention's key/value and
+    # query/gate projections over the 5120-wide hidden state; every projection's x is drawn,
+    # the multi-output GEMV uses the first one's
+    "attn_kv": ([("k", 1024, 5120, False), ("v", 1024, 5120, False)], 5, (1, 8)),
+    "attn_qgate": ([("q", 6144, 5120, False), ("gate", 6144, 5120, False)], 6, (1, 8)),
 }
 
 WORKLOADS = tuple(_RECIPES)

@@ -28,7 +28,7 @@ def L():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for required in ("nvfp4_pack_info", "nvfp4_gemv", "nvfp4_gemv_dual",
+    for required in ("nvfp4_pack_info", "nvfp4_gemv", "nvfp4_gemv_dual", "nvfp4_gemv_multi",
                      "nvfp4_workspace_bytes", "nvfp4_status_string"):
         assert required in names
 
@@ -128,3 +128,53 @@ def test_noalloc_host_checks(L):
     assert L.nvfp4_gemv_noalloc(A16, A16, 1.0, A16, 64, A16, 64, 0, 64, 64, None) == 0
     if not cuda_ok():
         assert L.nvfp4_gemv_noalloc(A16, A16, 1.0, A16, 64, A16, 64, 1, 64, 64, None) == -5
+
+
+def _outputs(*specs):
+    """nvfp4_output_t array from (w, s, g, y, ldy, n) tuples."""
+    arr = (nv.Output * len(specs))()
+    for o, (w, s, g, y, ldy, n) in enumerate(specs):
+        arr[o].w, arr[o].s, arr[o].global_scale = w, s, g
+        arr[o].y, arr[o].ldy, arr[o].n = y, ldy, n
+    return arr
+
+
+def test_multi_host_checks(L):
+    good = (A16, A16, 1.0, A16, 64, 64)
+    ok2 = _outputs(good, good)
+    # count out of range, descriptor array missing
+    assert L.nvfp4_gemv_multi(ok2, 0, A16, 64, 1, 64, A16, 1 << 30, 0, None) == -2
+    assert L.nvfp4_gemv_multi(_outputs(*[good] * 5), 5, A16, 64, 1, 64, A16, 1 << 30, 0,
+                              None) == -2
+    assert L.nvfp4_gemv_multi(None, 1, A16, 64, 1, 64, A16, 1 << 30, 0, None) == -1
+    # every output is vetted like nvfp4_gemv: rows, alignment, null weight, ldy < n, flags
+    assert L.nvfp4_gemv_multi(ok2, 2, A16, 64, 9, 64, A16, 1 << 30, 0, None) == -3
+    assert L.nvfp4_gemv_multi(_outputs(good, (A16 + 4, A16, 1.0, A16, 64, 64)), 2, A16, 64, 1,
+                              64, A16, 1 << 30, 0, None) == -4
+    assert L.nvfp4_gemv_multi(_outputs(good, (None, A16, 1.0, A16, 64, 64)), 2, A16, 64, 1, 64,
+                              A16, 1 << 30, 0, None) == -1
+    assert L.nvfp4_gemv_multi(_outputs(good, (A16, A16, 1.0, A16, 32, 64)), 2, A16, 64, 1, 64,
+                              A16, 1 << 30, 0, None) == -2
+    assert L.nvfp4_gemv_multi(ok2, 2, A16, 64, 1, 64, A16, 1 << 30, 2, None) == -2
+    # nothing to do: M = 0, or every output empty
+    assert L.nvfp4_gemv_multi(ok2, 2, A16, 64, 0, 64, A16, 1 << 30, 0, None) == 0
+    empty = (A16, A16, 1.0, A16, 64, 0)
+    assert L.nvfp4_gemv_multi(_outputs(empty, empty), 2, A16, 64, 1, 64, A16, 1 << 30, 0,
+                              None) == 0
+    if not cuda_ok():
+        assert L.nvfp4_gemv_multi(ok2, 2, A16, 64, 1, 64, A16, 1 << 30, 0, None) == -5
+
+
+def test_multi_binding_argument_checks():
+    import torch
+    w = torch.zeros((64, 32), dtype=torch.uint8)
+    s = torch.zeros((64, 4), dtype=torch.uint8)
+    x = torch.zeros((1, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        nv.gemv_multi([], x)
+    with pytest.raises(ValueError):
+        nv.gemv_multi([(w, s, 1.0)] * 5, x)
+    w2 = torch.zeros((64, 16), dtype=torch.uint8)
+    s2 = torch.zeros((64, 2), dtype=torch.uint8)
+    with pytest.raises(ValueError):  # K differs between outputs
+        nv.gemv_multi([(w, s, 1.0), (w2, s2, 1.0)], x)
