@@ -466,14 +466,18 @@ def run_ours(args, world, rank, local):
 
 
 def run_e2e(args, wl, dw, ws, world):
-    """Same metric through the public Python API (`gemv`, `gemv_dual`).  Every step copies the
-    step's inputs (each projection's x, 8 rows) from pinned host memory to the device in one
-    copy, runs the 64 calls, and reads every call's y back into pinned host memory in one copy;
-    both copies are inside the timed region."""
+    """Same metric through the public Python API (`gemv`, `gemv_dual`), as a serving loop runs
+    it.  Every step copies the step's inputs (each projection's x, 8 rows) from pinned host
+    memory to the device in one copy, runs the 64 calls, and reads every call's y back into
+    pinned host memory in one copy; all of it is inside the timed region.  The copies run on
+    their own streams (one for H2D, one for D2H) with two buffers, so one step's copies overlap
+    the neighbouring steps' kernels; events keep every buffer from being overwritten while a
+    copy or kernel still uses it."""
     import torch
     import nvfp4_weight_only_03_b200 as nv
     dev = dw[0]["x"].device
-    # one pinned host buffer and one device buffer for all x, one each for all y of the step
+    # one pinned host buffer of all x; two device buffers of all x and of all y, two pinned
+    # host buffers of all y (step i uses buffer i % 2)
     x_off, off = {}, 0
     for e in dw:
         x_off[e["p"].name] = off
@@ -483,55 +487,83 @@ def run_e2e(args, wl, dw, ws, world):
         o = x_off[e["p"].name]
         hx[o:o + e["x"].numel()].copy_(torch.from_numpy(e["p"].x.view(np.int16)).view(torch.bfloat16)
                                        .reshape(-1))
-    dx = torch.empty(off, dtype=torch.bfloat16, device=dev)
+    dx = [torch.empty(off, dtype=torch.bfloat16, device=dev) for _ in range(2)]
     y_off, off = {}, 0
     for m in wl.rows:
         for e in dw:
             y_off[(e["p"].name, m)] = off
             off += m * e["p"].n
-    hy = torch.empty(off, dtype=torch.bfloat16).pin_memory()
-    dy = torch.empty(off, dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream()
-    calls = []
-    for m in wl.rows:
-        for e in dw:
-            p = e["p"]
-            xo = x_off[p.name]
-            x = dx[xo:xo + 8 * p.k].view(8, p.k)[:m]
-            yo = y_off[(p.name, m)]
-            y = dy[yo:yo + m * p.n].view(m, p.n)
-            calls.append((e, x, y))
+    hy = [torch.empty(off, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    dy = [torch.empty(off, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    compute = torch.cuda.Stream(device=dev)
+    h2d = torch.cuda.Stream(device=dev)
+    d2h = torch.cuda.Stream(device=dev)
+    calls = [[], []]
+    for buf in range(2):
+        for m in wl.rows:
+            for e in dw:
+                p = e["p"]
+                xo = x_off[p.name]
+                x = dx[buf][xo:xo + 8 * p.k].view(8, p.k)[:m]
+                yo = y_off[(p.name, m)]
+                y = dy[buf][yo:yo + m * p.n].view(m, p.n)
+                calls[buf].append((e, x, y))
+    x_ready = [torch.cuda.Event() for _ in range(2)]    # H2D of buffer b done
+    x_free = [torch.cuda.Event() for _ in range(2)]     # kernels reading dx[b] done
+    y_ready = [torch.cuda.Event() for _ in range(2)]    # kernels writing dy[b] done
+    y_free = [torch.cuda.Event() for _ in range(2)]     # D2H of dy[b] done
+    for b in range(2):  # every buffer starts free
+        x_free[b].record(compute)
+        y_free[b].record(d2h)
 
-    def step():
-        dx.copy_(hx, non_blocking=True)
-        for e, x, y in calls:
-            if e["p"].dual:
-                nv.gemv_dual(e["W"], e["S"], e["g"], e["Wu"], e["Su"], e["gu"], x, y=y, ws=ws,
-                             stream=stream, prefetch_weights=True)
-            else:
-                nv.gemv(e["W"], e["S"], e["g"], x, y=y, ws=ws, stream=stream,
-                        prefetch_weights=True)
-        hy.copy_(dy, non_blocking=True)
+    def step(i):
+        b = i % 2
+        with torch.cuda.stream(h2d):
+            h2d.wait_event(x_free[b])
+            dx[b].copy_(hx, non_blocking=True)
+            x_ready[b].record(h2d)
+        with torch.cuda.stream(compute):
+            compute.wait_event(x_ready[b])
+            compute.wait_event(y_free[b])
+            for e, x, y in calls[b]:
+                if e["p"].dual:
+                    nv.gemv_dual(e["W"], e["S"], e["g"], e["Wu"], e["Su"], e["gu"], x, y=y, ws=ws,
+                                 stream=compute, prefetch_weights=True)
+                else:
+                    nv.gemv(e["W"], e["S"], e["g"], x, y=y, ws=ws, stream=compute,
+                            prefetch_weights=True)
+            x_free[b].record(compute)
+            y_ready[b].record(compute)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(y_ready[b])
+            hy[b].copy_(dy[b], non_blocking=True)
+            y_free[b].record(d2h)
 
-    for _ in range(3):
-        step()
+    for i in range(3):
+        step(i)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    t0.record(stream)
-    for _ in range(args.e2e_steps):
-        step()
-    t1.record(stream)
+    t0.record(h2d)  # the first H2D follows t0; the other streams wait for it too
+    compute.wait_event(t0)
+    d2h.wait_event(t0)
+    for i in range(args.e2e_steps):
+        step(i)
+    # the last D2H is the last piece of work; every stream ends before t1
+    d2h.wait_stream(compute)
+    d2h.wait_stream(h2d)
+    t1.record(d2h)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(t0.elapsed_time(t1), world)
     bytes_step = sum(step_bytes(wl).values())
     return {"value": round(world * bytes_step * args.e2e_steps / (ms * 1e-3) / 1e9, 1),
             "unit": "GB/s", "h2d_bytes_per_step": hx.numel() * 2,
-            "d2h_bytes_per_step": hy.numel() * 2, "steps": args.e2e_steps,
+            "d2h_bytes_per_step": hy[0].numel() * 2, "steps": args.e2e_steps,
             "api": "nvfp4_weight_only_03_b200.gemv / gemv_dual, one H2D copy of the step's x "
-                   "and one D2H copy of its y per step"}
+                   "and one D2H copy of its y per step, copies on their own streams overlapping "
+                   "the neighbouring steps (two buffers)"}
 
 
 # ----------------------------------------------------------------------------------------------
