@@ -9,11 +9,12 @@ Metric: effective HBM GB/s = (packed weights + scales + bf16 activations + bf16 
 per step / device time per step.  Printed as one JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload sweep|attn_pairs]
+                  [--workload sweep|attn_pairs|wide_rows]
 
 --workload attn_pairs measures nvfp4_gemv_multi instead: 8 layers x {k + v (2 x 1024x5120),
 q + gate (2 x 6144x5120)}, one launch per pair sharing x, M in {1, 8}; the same outputs as
-separate nvfp4_gemv launches are timed beside it.
+separate nvfp4_gemv launches are timed beside it.  --workload wide_rows times the sweep's first
+layer at M = 16, 32, 64 and 128 rows (one kernel pass per 8 rows).
 
 Under torchrun (N > 1) every rank runs an independent replica on its own GPU (the GEMV needs no
 collective); value = bytes of all ranks / max over ranks of the device time.
@@ -51,7 +52,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("sweep", "attn_pairs"), default="sweep")
+    ap.add_argument("--workload", choices=("sweep", "attn_pairs", "wide_rows"), default="sweep")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -807,6 +808,96 @@ def run_pairs(args, world, rank, local):
     return line
 
 
+# ----------------------------------------------------------------------------------------------
+# more than 8 rows (one kernel pass per 8-row block)
+
+WIDE_ROWS = (16, 32, 64, 128)
+WIDE_DESC = ("sweep layer 0 {qkv 10240x5120, o 5120x6144, gate_up dual 2x17408x5120, down "
+             "5120x17408} NVFP4 at M in {16,32,64,128} rows, one kernel pass per 8 rows, back to "
+             "back on one stream; value at M = 128")
+
+
+def run_wide(args, world, rank, local):
+    import torch
+    import nvfp4_weight_only_03_b200 as nv
+    L = nv.lib()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = synth.make(WORKLOAD, generate_x=False)
+    projs = wl.projections[:4]
+    ents = []
+    for i, p in enumerate(projs):
+        e = {"p": p, "W": torch.from_numpy(p.w.packed).to(dev), "S": torch.from_numpy(p.w.scales).to(dev),
+             "x": torch.from_numpy(synth.activations(wl.seed + 100, 2 * i * 128 * p.k, 128, p.k)
+                                   .view(np.int16)).view(torch.bfloat16).to(dev),
+             "y": torch.empty((128, p.n), dtype=torch.bfloat16, device=dev)}
+        if p.dual:
+            e["Wu"] = torch.from_numpy(p.w_up.packed).to(dev)
+            e["Su"] = torch.from_numpy(p.w_up.scales).to(dev)
+        ents.append(e)
+    ws = nv.workspace(dev)
+    stream = torch.cuda.Stream(device=dev)
+    flags = nv.FLAG_PREFETCH_WEIGHTS
+    per_m = {}
+    for m in WIDE_ROWS:
+        def launches(h):
+            for e in ents:
+                p = e["p"]
+                if p.dual:
+                    st = L.nvfp4_gemv_dual_ex(e["W"].data_ptr(), e["S"].data_ptr(), ctypes.c_float(p.w.g),
+                                              e["Wu"].data_ptr(), e["Su"].data_ptr(), ctypes.c_float(p.w_up.g),
+                                              e["x"].data_ptr(), p.k, e["y"].data_ptr(), p.n, m, p.n, p.k,
+                                              ws.data_ptr(), ws.numel(), flags, h)
+                else:
+                    st = L.nvfp4_gemv_ex(e["W"].data_ptr(), e["S"].data_ptr(), ctypes.c_float(p.w.g),
+                                         e["x"].data_ptr(), p.k, e["y"].data_ptr(), p.n, m, p.n, p.k,
+                                         ws.data_ptr(), ws.numel(), flags, h)
+                if st != 0:
+                    raise RuntimeError(f"launch failed: {nv.STATUS.get(st, st)}")
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 3)):
+                launches(stream.cuda_stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            launches(torch.cuda.current_stream().cuda_stream)
+        g.replay()
+        torch.cuda.synchronize()
+        steps = max(1, args.steps // m)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            t0.record()
+            for _ in range(steps):
+                g.replay()
+            t1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = max_over_ranks(t0.elapsed_time(t1), world) / steps
+        b = sum((2 if e["p"].dual else 1) * (e["p"].n * e["p"].k * 9 // 16) + m * e["p"].k * 2
+                + m * e["p"].n * 2 for e in ents)
+        fl = sum((2 if e["p"].dual else 1) * 2 * m * e["p"].n * e["p"].k for e in ents)
+        per_m[m] = {"ms_per_step": round(ms, 5), "GBps": round(world * b / (ms * 1e-3) / 1e9, 1),
+                    "TFLOPs": round(world * fl / (ms * 1e-3) / 1e12, 1), "steps": steps,
+                    "launches_per_step": 4 * ((m + 7) // 8)}
+        del g
+    peak, peak_src = peaks()
+    top = per_m[WIDE_ROWS[-1]]
+    return {"metric": METRIC, "value": top["GBps"], "unit": "GB/s", "n_gpus": world,
+            "steps": top["steps"], "warmup": args.warmup, "ms_per_step": top["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4(e2m1+e4m3) x bf16 -> fp32 accumulate, bf16 out",
+            "data": "synthetic (seeded N(0,0.02) weights quantised to NVFP4, N(0,1) bf16 x)",
+            "config": {"workload": WIDE_DESC, "rows": list(WIDE_ROWS),
+                       "l2": "0.2 GB of weights per pass, no flush; passes after the first of a "
+                             "call find part of the weights in L2"},
+            "roofline": {"bound": "hbm", "achieved": top["GBps"], "peak": peak, "unit": "GB/s",
+                         "frac": round(top["GBps"] / peak, 4), "traffic": None,
+                         "peak_source": peak_src,
+                         "note": "algorithmic bytes count the weights once per call"},
+            "per_rows": per_m, "gpu_launches": top["launches_per_step"] * top["steps"]}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -817,7 +908,8 @@ def main():
             print(json.dumps(line), flush=True)
         return
     world, rank, local = dist_setup(args.gpus)
-    line = (run_pairs if args.workload == "attn_pairs" else run_ours)(args, world, rank, local)
+    run = {"sweep": run_ours, "attn_pairs": run_pairs, "wide_rows": run_wide}[args.workload]
+    line = run(args, world, rank, local)
     if line is not None and rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -7,7 +7,10 @@
  * "nvfp4/g16" and bf16 activations ("Blueprint - circuit executor" page for
  * qwen3.8-27b-nvfp4 on GB10, tables "Kernels the plan launches" and "Weighted nodes").
  * Row counts 1 (plain decode) to 8 (an 8-row speculative draft/verify round, kern-qwen38-sm103
- * model card, section "Run"; NInfer card, DFlash2 "block width 8").
+ * model card, section "Run"; NInfer card, DFlash2 "block width 8"), and up to 128 for the plan's
+ * wider arms (multi_seq rows 2..128, same page, table "Plan arms").  One kernel pass computes
+ * up to NVFP4_PASS_ROWS = 8 rows; a call with more rows runs ceil(M/8) passes over consecutive
+ * 8-row blocks, each pass streaming the weights again (mostly from L2 when they fit there).
  *
  * Storage layout (layout_version 1):
  *   W  uint8 [N][K/2]   byte b of row n holds element k = 2b in bits 0..3 and k = 2b+1 in
@@ -27,9 +30,9 @@
  * in fp32 -- the SiLU(gate)*up that the GB10 plan runs as a separate "moe_silu_mul" launch.
  *
  * Guarantees:
- *   - Row invariance: output row m is bitwise identical for every M in 1..8 given the same
+ *   - Row invariance: output row m is bitwise identical for every M in 1..128 given the same
  *     x row, weights, N, K and device (the kernel's work split depends on N, K and the SM
- *     count, never on M).
+ *     count, never on M, and a row's arithmetic depends only on that row).
  *   - Determinism: identical calls give bitwise identical results.
  *
  * Conventions (every entry point):
@@ -60,14 +63,15 @@ typedef enum {
     NVFP4_OK = 0,
     NVFP4_ERR_NULL = -1,      /* a required pointer is NULL */
     NVFP4_ERR_SHAPE = -2,     /* N < 0, K < 0, K % 32 != 0, ldx < K, ldy < N, K too large */
-    NVFP4_ERR_ROWS = -3,      /* M < 0 or M > 8 */
+    NVFP4_ERR_ROWS = -3,      /* M < 0 or M > NVFP4_MAX_ROWS (128) */
     NVFP4_ERR_ALIGN = -4,     /* pointer or stride alignment (see each call) */
     NVFP4_ERR_ARCH = -5,      /* current device is not compute capability 10.0 (B200) */
     NVFP4_ERR_LAUNCH = -6,    /* the CUDA launch failed (cudaGetLastError) */
     NVFP4_ERR_WORKSPACE = -7  /* workspace NULL, misaligned or smaller than required */
 } nvfp4_status;
 
-#define NVFP4_MAX_ROWS 8
+#define NVFP4_MAX_ROWS 128 /* rows of x (and y) per call */
+#define NVFP4_PASS_ROWS 8  /* rows one kernel pass computes; more run as ceil(M/8) passes */
 #define NVFP4_MAX_OUTPUTS 4
 #define NVFP4_GROUP 16
 #define NVFP4_LAYOUT_VERSION 1
@@ -88,7 +92,7 @@ typedef struct {
     int64_t weight_row_bytes; /* K/2    */
     int64_t scale_row_bytes;  /* K/16   */
     int32_t group;            /* 16 */
-    int32_t max_rows;         /* 8 */
+    int32_t max_rows;         /* 128 (NVFP4_MAX_ROWS) */
     int32_t align_bytes;      /* 16: required alignment of W and x */
     int32_t layout_version;   /* 1 */
 } nvfp4_pack_info_t;
@@ -106,7 +110,7 @@ int nvfp4_workspace_bytes(size_t* bytes);
 /* y = W x (single output), see the header comment.
  *   w, x: 16-byte aligned;  s, y: 2-byte aligned;  workspace: 16-byte aligned, at least
  *   nvfp4_workspace_bytes() bytes, zero-filled before first use.
- *   ldx % 8 == 0, ldx >= K;  ldy >= N.  1 <= M <= 8 (M == 0 and N == 0 are no-ops);
+ *   ldx % 8 == 0, ldx >= K;  ldy >= N.  1 <= M <= 128 (M == 0 and N == 0 are no-ops);
  *   K % 32 == 0 (K == 0 writes zeros).
  * Enqueued on `stream`; returns NVFP4_OK or an nvfp4_status error (nothing is enqueued on
  * error). */
@@ -156,7 +160,7 @@ typedef struct {
  * every weight.  When K is so large that nvfp4_gemv itself would split an output's rows over
  * several launches, and the outputs together exceed one launch, each output runs as its own
  * nvfp4_gemv_ex call instead.  Either way each result depends only on (every output's n, K,
- * SM count) and x's row: row invariance over M = 1..8 and determinism hold as for nvfp4_gemv,
+ * SM count) and x's row: row invariance over M = 1..128 and determinism hold as for nvfp4_gemv,
  * and the result of an output alone (count 1) is bitwise that of nvfp4_gemv_ex.  Output
  * buffers must not overlap one another, x or the weights.
  * Errors: NVFP4_ERR_NULL (outputs NULL, or as nvfp4_gemv for an output), NVFP4_ERR_SHAPE

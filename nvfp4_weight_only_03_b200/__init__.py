@@ -10,7 +10,8 @@ missing or the device is not a B200 the calls raise.
     k_, v_ = gemv_multi([(wk, sk, gk), (wv, sv, gv)], x)  # several outputs sharing x, one pass
 
 w: uint8 [N][K/2] packed e2m1 (low nibble = even k), s: uint8 [N][K/16] e4m3 scale codes,
-g: float global scale, x: bfloat16 [M][K] (M = 1..8, row stride may exceed K).
+g: float global scale, x: bfloat16 [M][K] (M = 1..128, one kernel pass per 8 rows; row stride
+may exceed K).
 """
 from __future__ import annotations
 
@@ -27,7 +28,8 @@ _lib = None
 STATUS = {0: "NVFP4_OK", -1: "NVFP4_ERR_NULL", -2: "NVFP4_ERR_SHAPE", -3: "NVFP4_ERR_ROWS",
           -4: "NVFP4_ERR_ALIGN", -5: "NVFP4_ERR_ARCH", -6: "NVFP4_ERR_LAUNCH",
           -7: "NVFP4_ERR_WORKSPACE"}
-MAX_ROWS = 8
+MAX_ROWS = 128
+PASS_ROWS = 8
 MAX_OUTPUTS = 4
 GROUP = 16
 FLAG_PREFETCH_WEIGHTS = 1

@@ -839,7 +839,7 @@ template <bool DUAL>
 int64_t max_groups_per_launch(int64_t k, int sms) {
     using C = Cfg<DUAL>;
     const int ku = (int)((k + kUnitK - 1) / kUnitK);
-    const size_t mx = NVFP4_MAX_ROWS;
+    const size_t mx = NVFP4_PASS_ROWS;
     const int64_t max_slots = (int64_t)((kSmemMax - 1024 - kMinStages * C::kStageBytes -
                                          mx * kRowPadU4 * 16) /
                                         (mx * kXSlotBytes));
@@ -856,6 +856,24 @@ int launch_spans(const Span* sp, int count, const void* x, int64_t ldx, int m, i
     using C = Cfg<DUAL>;
     static_assert(!(DUAL && MULTI), "the dual kernel has one output");
     if (count > Maps<DUAL, MULTI>::kCount / (DUAL ? 2 : 1)) return NVFP4_ERR_SHAPE;
+    if (m > NVFP4_PASS_ROWS) {
+        // more rows than one pass: consecutive blocks of NVFP4_PASS_ROWS rows of x and y, one
+        // launch each, in stream order on the same workspace; every row is computed exactly
+        // as in a call of its own block, so rows stay bitwise invariant over M
+        for (int r0 = 0; r0 < m; r0 += NVFP4_PASS_ROWS) {
+            Span part[kMaxOutputs];
+            for (int o = 0; o < count; ++o) {
+                part[o] = sp[o];
+                part[o].y = static_cast<uint16_t*>(sp[o].y) + (int64_t)r0 * sp[o].ldy;
+            }
+            const int rows = m - r0 < NVFP4_PASS_ROWS ? m - r0 : NVFP4_PASS_ROWS;
+            const int st = launch_spans<DUAL, MULTI>(
+                part, count, static_cast<const uint16_t*>(x) + (int64_t)r0 * ldx, ldx, rows, k,
+                ws, ws_bytes, flags, stream);
+            if (st != NVFP4_OK) return st;
+        }
+        return NVFP4_OK;
+    }
     constexpr int NS = C::kStreams;
     int dev = 0;
     DeviceInfo* di = nullptr;

@@ -54,7 +54,7 @@ def test_pack_info():
     assert info["weight_bytes"] == 10240 * 2560
     assert info["scale_bytes"] == 10240 * 320
     assert info["weight_row_bytes"] == 2560 and info["scale_row_bytes"] == 320
-    assert info["group"] == 16 and info["max_rows"] == 8
+    assert info["group"] == 16 and info["max_rows"] == 128
     assert info["align_bytes"] == 16 and info["layout_version"] == 1
     for bad in ((10, 48), (-1, 32), (4, -32)):
         with pytest.raises(nv.Nvfp4Error) as e:
@@ -87,7 +87,7 @@ def call_dual(L, m=1, n=64, k=64, wu=A16, su=A16, **kw):
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(m=9), -3), (dict(m=-1), -3),
+    (dict(m=129), -3), (dict(m=-1), -3),
     (dict(k=48), -2), (dict(k=-32), -2), (dict(n=-1), -2),
     (dict(ldx=32), -2), (dict(ldy=10), -2),
     (dict(w=None), -1), (dict(s=None), -1), (dict(x=None), -1), (dict(y=None), -1),
@@ -110,7 +110,7 @@ def test_dual_host_checks(L):
                              1 << 30, None) == -1
     assert L.nvfp4_gemv_dual(A16, A16, 1.0, A16 + 4, A16, 1.0, A16, 64, A16, 64, 1, 64, 64,
                              A16, 1 << 30, None) == -4
-    assert L.nvfp4_gemv_dual(A16, A16, 1.0, A16, A16, 1.0, A16, 64, A16, 64, 10, 64, 64, A16,
+    assert L.nvfp4_gemv_dual(A16, A16, 1.0, A16, A16, 1.0, A16, 64, A16, 64, 130, 64, 64, A16,
                              1 << 30, None) == -3
 
 
@@ -122,7 +122,7 @@ def test_valid_call_without_device_reports_arch(L):
 
 
 def test_noalloc_host_checks(L):
-    assert L.nvfp4_gemv_noalloc(A16, A16, 1.0, A16, 64, A16, 64, 9, 64, 64, None) == -3
+    assert L.nvfp4_gemv_noalloc(A16, A16, 1.0, A16, 64, A16, 64, 129, 64, 64, None) == -3
     assert L.nvfp4_gemv_noalloc(A16, A16, 1.0, A16 + 8, 64, A16, 64, 1, 64, 64, None) == -4
     assert L.nvfp4_gemv_noalloc(None, A16, 1.0, A16, 64, A16, 64, 1, 64, 64, None) == -1
     assert L.nvfp4_gemv_noalloc(A16, A16, 1.0, A16, 64, A16, 64, 0, 64, 64, None) == 0
@@ -148,7 +148,7 @@ def test_multi_host_checks(L):
                               None) == -2
     assert L.nvfp4_gemv_multi(None, 1, A16, 64, 1, 64, A16, 1 << 30, 0, None) == -1
     # every output is vetted like nvfp4_gemv: rows, alignment, null weight, ldy < n, flags
-    assert L.nvfp4_gemv_multi(ok2, 2, A16, 64, 9, 64, A16, 1 << 30, 0, None) == -3
+    assert L.nvfp4_gemv_multi(ok2, 2, A16, 64, 129, 64, A16, 1 << 30, 0, None) == -3
     assert L.nvfp4_gemv_multi(_outputs(good, (A16 + 4, A16, 1.0, A16, 64, 64)), 2, A16, 64, 1,
                               64, A16, 1 << 30, 0, None) == -4
     assert L.nvfp4_gemv_multi(_outputs(good, (None, A16, 1.0, A16, 64, 64)), 2, A16, 64, 1, 64,

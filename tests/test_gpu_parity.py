@@ -293,7 +293,7 @@ def test_error_statuses_on_device(ws):
                         o.get("ldy", 64), o.get("m", 1), 64, 64, o.get("ws", ws.data_ptr()),
                         o.get("wsb", ws.numel()), None)
     assert L.nvfp4_gemv(*args()) == 0
-    assert L.nvfp4_gemv(*args(m=9)) == -3
+    assert L.nvfp4_gemv(*args(m=129)) == -3
     assert L.nvfp4_gemv(*args(x=x.data_ptr() + 2)) == -4
     assert L.nvfp4_gemv(*args(w=W.data_ptr() + 1)) == -4
     assert L.nvfp4_gemv(*args(wsb=1024)) == -7

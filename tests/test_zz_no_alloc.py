@@ -92,6 +92,6 @@ def test_rejects_bad_arguments_before_launch():
     h = torch.cuda.current_stream().cuda_stream
     buf = torch.zeros(4096, dtype=torch.uint8, device="cuda")
     p = buf.data_ptr()
-    assert L.nvfp4_gemv_noalloc(p, p, 1.0, p, 64, p, 64, 9, 64, 64, h) == -3
+    assert L.nvfp4_gemv_noalloc(p, p, 1.0, p, 64, p, 64, 129, 64, 64, h) == -3
     assert L.nvfp4_gemv_noalloc(p, p, 1.0, p + 8, 64, p, 64, 1, 64, 64, h) == -4
     assert L.nvfp4_gemv_noalloc(p, p, 1.0, p, 64, p, 64, 1, 64, 48, h) == -2
