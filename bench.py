@@ -65,12 +65,12 @@ def parse():
 # launch, for layer 0 of the sweep at M = 1 and M = 8 (profiles/nvfp4_gemv_sweep_dram_traffic.md).
 # They describe the kernel code with this SHA-256 only (kernel_code_sha256: comments and blank
 # lines do not count); for any other code the bench reports traffic as null.
-TRAFFIC_SOURCE_SHA256 = "74d3718b9e3f2858f9477ad77e83e5b0a65abaf2aa307e6c7b4fb1efe1750535"
+TRAFFIC_SOURCE_SHA256 = "aad8d5a4ede9c0a2f49e9b26837381cdb8f7687bd8642ebfa62c2de57c4b349e"
 TRAFFIC_BYTES = {
-    ("L0.qkv", 1): 30118656, ("L0.o", 1): 18324224, ("L0.gate_up", 1): 107017472,
-    ("L0.down", 1): 50821888,
-    ("L0.qkv", 8): 29616896, ("L0.o", 8): 17837056, ("L0.gate_up", 8): 105765376,
-    ("L0.down", 8): 50488576,
+    ("L0.qkv", 1): 30119168, ("L0.o", 1): 18324480, ("L0.gate_up", 1): 106633472,
+    ("L0.down", 1): 50805760,
+    ("L0.qkv", 8): 29617408, ("L0.o", 8): 17837056, ("L0.gate_up", 8): 106331392,
+    ("L0.down", 8): 50459392,
 }
 KERNEL_SOURCE = os.path.join(ROOT, "nvfp4_weight_only_03_b200", "csrc", "nvfp4_gemv.cu")
 
