@@ -1,11 +1,15 @@
-// Weight-only NVFP4 GEMV / fused dual GEMV for NVIDIA B200 (sm_100a), with its C ABI.
+// Weight-only NVFP4 GEMV / fused dual GEMV / multi-output GEMV for NVIDIA B200 (sm_100a), with
+// its C ABI.
 //
 // The operation is the "w4a16_gemv" / "w4a16_gemv_dual" kernel family of a hybrid decoder's
 // decode step ("Blueprint - circuit executor" page for qwen3.8-27b-nvfp4 on GB10, table
 // "Kernels the plan launches"; weight format "nvfp4/g16", activations bf16, table "Weighted
 // nodes"); the fused SiLU(gate)*up epilogue replaces that plan's separate "moe_silu_mul" launch
-// (planner setting decode_split_silu).  Row counts 1..8 (8-row speculative draft/verify round,
-// kern-qwen38-sm103 model card, section "Run").  Formats and the ABI are described in nvfp4.h.
+// (planner setting decode_split_silu).  The multi-output instance runs up to four weights that
+// share x in one launch (that plan's two-output k/v and q+gate GEMVs).  Row counts 1..8 per pass
+// (8-row speculative draft/verify round, kern-qwen38-sm103 model card, section "Run"); calls of
+// up to 128 rows (the plan's multi_seq arms) run one pass per 8 rows.  Formats and the ABI are
+// described in nvfp4.h.
 //
 // Design (B200-first):
 //   * The path is HBM-bound: 0.5625 bytes per weight.  A persistent grid (one CTA per SM)
@@ -27,7 +31,8 @@
 //   * The dot products run on the tensor cores: mma.m16n8k16 (f16 in, fp32 accumulate) with
 //     16 weight rows as A and x as B, padded to 8 columns (columns >= M are zero).  The same
 //     instruction sequence serves every M, so row m of the output depends only on x row m:
-//     bitwise row invariance across M = 1..8.  Within a 16-row tile the mma's row r is weight
+//     bitwise row invariance across M = 1..8, and across 1..128 with the 8-row passes.  Within a
+//     16-row tile the mma's row r is weight
 //     row perm(r) (rows r and r+1 four apart), which makes the swizzled reads conflict-free.
 //   * x is staged once per CTA in shared memory as f16 (cp.async, then converted in place,
 //     each row by its own warps).  Each x row m is scaled by a power of two 2^e(m) chosen from
