@@ -33,6 +33,7 @@ PASS_ROWS = 8
 MAX_OUTPUTS = 4
 GROUP = 16
 FLAG_PREFETCH_WEIGHTS = 1
+FLAG_WIDE_TENSOR = 2
 
 
 class Nvfp4Error(RuntimeError):
@@ -83,11 +84,12 @@ def lib():
         L.nvfp4_gemv_multi.argtypes = [ctypes.POINTER(Output), c_int, vp, i64, c_int, i64, vp,
                                        sz, ctypes.c_uint32, vp]
         L.nvfp4_workspace_error.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
+        L.nvfp4_workspace_bytes_wide.argtypes = [i64, i64, c_int, ctypes.POINTER(sz)]
         L.nvfp4_status_string.argtypes = [c_int]
         L.nvfp4_status_string.restype = ctypes.c_char_p
         for f in (L.nvfp4_pack_info, L.nvfp4_workspace_bytes, L.nvfp4_gemv, L.nvfp4_gemv_dual,
                   L.nvfp4_gemv_ex, L.nvfp4_gemv_dual_ex, L.nvfp4_gemv_noalloc,
-                  L.nvfp4_gemv_multi, L.nvfp4_workspace_error):
+                  L.nvfp4_gemv_multi, L.nvfp4_workspace_error, L.nvfp4_workspace_bytes_wide):
             f.restype = c_int
         _lib = L
     return _lib
@@ -107,6 +109,12 @@ def pack_info(n: int, k: int) -> dict:
 def workspace_bytes() -> int:
     b = ctypes.c_size_t()
     _check(lib().nvfp4_workspace_bytes(ctypes.byref(b)), "nvfp4_workspace_bytes")
+    return int(b.value)
+
+
+def workspace_bytes_wide(n: int, k: int, m: int) -> int:
+    b = ctypes.c_size_t()
+    _check(lib().nvfp4_workspace_bytes_wide(n, k, m, ctypes.byref(b)), "nvfp4_workspace_bytes_wide")
     return int(b.value)
 
 
@@ -169,17 +177,39 @@ def _out(y, m, n, x):
     return y, y.stride(0) if m > 1 else n
 
 
+_wide_workspaces: dict = {}
+
+
+def wide_workspace(n: int, k: int, m: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace large enough for a wide_tensor call of this shape (cached per
+    device, grown when a larger one is needed)."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else
+                       torch.device(device).index or 0)
+    need = workspace_bytes_wide(n, k, m)
+    ws = _wide_workspaces.get(dev)
+    if ws is None or ws.numel() < need:
+        with torch.cuda.device(dev):
+            ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+        _wide_workspaces[dev] = ws
+    return ws
+
+
 def gemv(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor, y: torch.Tensor = None,
-         ws: torch.Tensor = None, stream=None, prefetch_weights: bool = False) -> torch.Tensor:
+         ws: torch.Tensor = None, stream=None, prefetch_weights: bool = False,
+         wide_tensor: bool = False) -> torch.Tensor:
     """y[m][n] = bf16(g * sum_k e2m1(w[n][k]) * e4m3(s[n][k/16]) * x[m][k]) on the GPU.
 
     prefetch_weights: stream w and s before earlier work on the stream has finished
-    (programmatic dependent launch); only valid when that work does not write w or s."""
+    (programmatic dependent launch); only valid when that work does not write w or s.
+    wide_tensor: calls of 9..128 rows run on the tensor-core tier (one pass over the weights;
+    rows invariant over 9..128, equal to 1..8-row calls within the tolerance)."""
     n, k = _weight_args(w, s)
     x, m, ldx = _x_args(x, k)
     y, ldy = _out(y, m, n, x)
-    ws = workspace(x.device) if ws is None else ws
-    flags = FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0
+    if ws is None:
+        ws = wide_workspace(n, k, m, x.device) if wide_tensor else workspace(x.device)
+    flags = (FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0) | \
+        (FLAG_WIDE_TENSOR if wide_tensor else 0)
     st = lib().nvfp4_gemv_ex(w.data_ptr(), s.data_ptr(), float(g), x.data_ptr(), ldx,
                              y.data_ptr(), ldy, m, n, k, ws.data_ptr(), ws.numel(), flags,
                              _stream(stream))

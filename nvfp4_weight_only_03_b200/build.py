@@ -6,8 +6,8 @@ import subprocess
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SRC = os.path.join(HERE, "csrc", "nvfp4_gemv.cu")
-HDR = os.path.join(ROOT, "include", "nvfp4.h")
+SRCS = [os.path.join(HERE, "csrc", "nvfp4_gemv.cu"), os.path.join(HERE, "csrc", "nvfp4_gemv_tc.cu")]
+HDRS = [os.path.join(ROOT, "include", "nvfp4.h"), os.path.join(HERE, "csrc", "nvfp4_tc.h")]
 LIB = os.path.join(HERE, "libnvfp4gemv.so")
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -22,10 +22,10 @@ def nvcc() -> str:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    newest = max(os.path.getmtime(SRC), os.path.getmtime(HDR))
+    newest = max(os.path.getmtime(f) for f in SRCS + HDRS)
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < newest:
         tmp = LIB + f".tmp{os.getpid()}"
-        cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), SRC, "-o", tmp]
+        cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), *SRCS, "-o", tmp]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         subprocess.check_call(cmd)

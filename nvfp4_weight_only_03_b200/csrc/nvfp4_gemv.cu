@@ -53,6 +53,7 @@
 #include <string.h>
 
 #include "nvfp4.h"
+#include "nvfp4_tc.h"
 
 namespace {
 
@@ -787,7 +788,8 @@ bool misaligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t
 int check_common(const void* x, int64_t ldx, const void* y, int64_t ldy, int m, int64_t n,
                  int64_t k, const void* ws, uint32_t flags, bool* noop) {
     *noop = false;
-    if (flags & ~(uint32_t)NVFP4_FLAG_PREFETCH_WEIGHTS) return NVFP4_ERR_SHAPE;
+    if (flags & ~(uint32_t)(NVFP4_FLAG_PREFETCH_WEIGHTS | NVFP4_FLAG_WIDE_TENSOR))
+        return NVFP4_ERR_SHAPE;
     if (m < 0 || m > NVFP4_MAX_ROWS) return NVFP4_ERR_ROWS;
     if (n < 0 || k < 0 || (k % 32) != 0 || k > kMaxK) return NVFP4_ERR_SHAPE;
     if (m == 0 || n == 0) {
@@ -1079,6 +1081,16 @@ int nvfp4_gemv_ex(const uint8_t* w, const uint8_t* s, float global_scale, const 
     int st = check_common(x, ldx, y, ldy, m, n, k, workspace, flags, &noop);
     if (st != NVFP4_OK || noop) return st;
     if (k > 0 && (st = check_weight(w, s)) != NVFP4_OK) return st;
+    if ((flags & NVFP4_FLAG_WIDE_TENSOR) && m > NVFP4_PASS_ROWS && k > 0 &&
+        nvfp4_tc::usable(s, k)) {
+        int dev = 0;
+        DeviceInfo* di = nullptr;
+        if ((st = device_info(&dev, &di)) != NVFP4_OK) return st;
+        size_t flags_off, partial_off;
+        const size_t base = workspace_layout(di->sms, &flags_off, &partial_off);
+        return nvfp4_tc::launch(g_encode, di->sms, w, s, global_scale, x, ldx, y, ldy, m, n, k,
+                                workspace, workspace_bytes, base, stream);
+    }
     const uint8_t* ws_[1] = {w};
     const uint8_t* ss_[1] = {s};
     const float gs[1] = {global_scale};
@@ -1204,6 +1216,20 @@ int nvfp4_gemv_multi(const nvfp4_output_t* outputs, int count, const void* x, in
                                 workspace_bytes, flags, stream)) != NVFP4_OK)
             return st;
     }
+    return NVFP4_OK;
+}
+
+int nvfp4_workspace_bytes_wide(int64_t n, int64_t k, int m, size_t* bytes) {
+    if (!bytes) return NVFP4_ERR_NULL;
+    if (n < 0 || k < 0 || (k % 32) != 0 || k > kMaxK) return NVFP4_ERR_SHAPE;
+    if (m < 0 || m > NVFP4_MAX_ROWS) return NVFP4_ERR_ROWS;
+    int dev = 0;
+    DeviceInfo* di = nullptr;
+    int st = device_info(&dev, &di);
+    if (st != NVFP4_OK) return st;
+    size_t flags_off, partial_off;
+    *bytes = workspace_layout(di->sms, &flags_off, &partial_off) +
+             (m > NVFP4_PASS_ROWS ? nvfp4_tc::scratch_bytes(n, k, m, di->sms) : 0);
     return NVFP4_OK;
 }
 

@@ -1,0 +1,32 @@
+// Internal interface of the tensor-core tier (nvfp4_gemv_tc.cu) for the C ABI in nvfp4_gemv.cu.
+#ifndef NVFP4_TC_H
+#define NVFP4_TC_H
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace nvfp4_tc {
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// K-splits of an N x K call (depends only on N, K and the SM count).
+int choose_splits(int64_t n, int64_t k, int sms);
+// Scratch bytes of a tier call of m rows: fp32 partials (when K is split), an f16 copy of x and
+// the rows' scales.
+size_t scratch_bytes(int64_t n, int64_t k, int m, int sms);
+// The tier's TMA scale boxes need K % 256 == 0 and 16-byte aligned scale codes.
+bool usable(const void* s, int64_t k);
+// Enqueue one call (arguments already checked as for nvfp4_gemv, 9 <= m <= 128).  The error
+// word is the workspace's first int32; the scratch starts scratch_off bytes in.
+int launch(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g, const void* x,
+           int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws,
+           size_t ws_bytes, size_t scratch_off, cudaStream_t stream);
+
+}  // namespace nvfp4_tc
+
+#endif

@@ -155,7 +155,7 @@ def test_multi_host_checks(L):
                               A16, 1 << 30, 0, None) == -1
     assert L.nvfp4_gemv_multi(_outputs(good, (A16, A16, 1.0, A16, 32, 64)), 2, A16, 64, 1, 64,
                               A16, 1 << 30, 0, None) == -2
-    assert L.nvfp4_gemv_multi(ok2, 2, A16, 64, 1, 64, A16, 1 << 30, 2, None) == -2
+    assert L.nvfp4_gemv_multi(ok2, 2, A16, 64, 1, 64, A16, 1 << 30, 4, None) == -2
     # nothing to do: M = 0, or every output empty
     assert L.nvfp4_gemv_multi(ok2, 2, A16, 64, 0, 64, A16, 1 << 30, 0, None) == 0
     empty = (A16, A16, 1.0, A16, 64, 0)
@@ -178,3 +178,19 @@ def test_multi_binding_argument_checks():
     s2 = torch.zeros((64, 2), dtype=torch.uint8)
     with pytest.raises(ValueError):  # K differs between outputs
         nv.gemv_multi([(w, s, 1.0), (w2, s2, 1.0)], x)
+
+
+def test_wide_tensor_flag_host_checks(L):
+    # the flag is accepted; an unknown bit is not
+    ex = lambda m, flags: L.nvfp4_gemv_ex(A16, A16, 1.0, A16, 64, A16, 64, m, 64, 64, A16,
+                                          1 << 30, flags, None)
+    assert ex(0, nv.FLAG_WIDE_TENSOR) == 0
+    assert ex(1, 4) == -2
+    if not cuda_ok():
+        assert ex(16, nv.FLAG_WIDE_TENSOR) == -5
+    b = ctypes.c_size_t()
+    assert L.nvfp4_workspace_bytes_wide(64, 64, 16, None) == -1
+    assert L.nvfp4_workspace_bytes_wide(64, 48, 16, ctypes.byref(b)) == -2
+    assert L.nvfp4_workspace_bytes_wide(64, 64, 129, ctypes.byref(b)) == -3
+    if not cuda_ok():
+        assert L.nvfp4_workspace_bytes_wide(64, 64, 16, ctypes.byref(b)) == -5
