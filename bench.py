@@ -65,12 +65,12 @@ def parse():
 # launch, for layer 0 of the sweep at M = 1 and M = 8 (profiles/nvfp4_gemv_sweep_dram_traffic.md).
 # They describe the kernel code with this SHA-256 only (kernel_code_sha256: comments and blank
 # lines do not count); for any other code the bench reports traffic as null.
-TRAFFIC_SOURCE_SHA256 = "aad8d5a4ede9c0a2f49e9b26837381cdb8f7687bd8642ebfa62c2de57c4b349e"
+TRAFFIC_SOURCE_SHA256 = "ee6c5010fb162609c1317241ee9af6bd097f7543628b6e1361b6027ffd8ccefa"
 TRAFFIC_BYTES = {
-    ("L0.qkv", 1): 30119168, ("L0.o", 1): 18324480, ("L0.gate_up", 1): 106633472,
-    ("L0.down", 1): 50805760,
-    ("L0.qkv", 8): 29617408, ("L0.o", 8): 17837056, ("L0.gate_up", 8): 106331392,
-    ("L0.down", 8): 50459392,
+    ("L0.qkv", 1): 30119168, ("L0.o", 1): 18324480, ("L0.gate_up", 1): 106838784,
+    ("L0.down", 1): 50807040,
+    ("L0.qkv", 8): 29617152, ("L0.o", 8): 17837568, ("L0.gate_up", 8): 108867328,
+    ("L0.down", 8): 50468864,
 }
 KERNEL_SOURCE = os.path.join(ROOT, "nvfp4_weight_only_03_b200", "csrc", "nvfp4_gemv.cu")
 
@@ -854,7 +854,7 @@ def run_wide(args, world, rank, local):
                          "unit": "TFLOP/s", "frac": round(top["TFLOPs"] / peaks_bf16()[0], 4),
                          "traffic": None, "peak_source": peaks_bf16()[1],
                          "note": "f16 tcgen05 MMAs against the measured bf16 cuBLAS burst peak "
-                                 "(the same rate for f16); the dual runs as 8-row passes"},
+                                 "(the same rate for f16); the dual runs both streams on the tier"},
             "per_rows": per_mode, "gpu_launches": None}
 
 

@@ -233,15 +233,21 @@ def gemv_noalloc(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor,
 
 def gemv_dual(wg: torch.Tensor, sg: torch.Tensor, gg: float, wu: torch.Tensor, su: torch.Tensor,
               gu: float, x: torch.Tensor, y: torch.Tensor = None, ws: torch.Tensor = None,
-              stream=None, prefetch_weights: bool = False) -> torch.Tensor:
-    """o[m][n] = bf16(silu(gate) * up), gate/up the two NVFP4 GEMVs of the same x."""
+              stream=None, prefetch_weights: bool = False,
+              wide_tensor: bool = False) -> torch.Tensor:
+    """o[m][n] = bf16(silu(gate) * up), gate/up the two NVFP4 GEMVs of the same x.
+
+    wide_tensor: calls of 9..128 rows run gate and up on the tensor-core tier, kept in fp32
+    and combined by one final pass."""
     n, k = _weight_args(wg, sg)
     if _weight_args(wu, su) != (n, k):
         raise ValueError("gate and up weights must have the same shape")
     x, m, ldx = _x_args(x, k)
     y, ldy = _out(y, m, n, x)
-    ws = workspace(x.device) if ws is None else ws
-    flags = FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0
+    if ws is None:
+        ws = wide_workspace(n, k, m, x.device) if wide_tensor else workspace(x.device)
+    flags = (FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0) | \
+        (FLAG_WIDE_TENSOR if wide_tensor else 0)
     st = lib().nvfp4_gemv_dual_ex(wg.data_ptr(), sg.data_ptr(), float(gg), wu.data_ptr(),
                                   su.data_ptr(), float(gu), x.data_ptr(), ldx, y.data_ptr(), ldy,
                                   m, n, k, ws.data_ptr(), ws.numel(), flags, _stream(stream))

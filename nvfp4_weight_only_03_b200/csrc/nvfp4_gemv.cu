@@ -1154,6 +1154,17 @@ int nvfp4_gemv_dual_ex(const uint8_t* w_gate, const uint8_t* s_gate, float globa
         if ((st = check_weight(w_gate, s_gate)) != NVFP4_OK) return st;
         if ((st = check_weight(w_up, s_up)) != NVFP4_OK) return st;
     }
+    if ((flags & NVFP4_FLAG_WIDE_TENSOR) && m > NVFP4_PASS_ROWS && k > 0 &&
+        nvfp4_tc::usable(s_gate, k) && nvfp4_tc::usable(s_up, k)) {
+        int dev = 0;
+        DeviceInfo* di = nullptr;
+        if ((st = device_info(&dev, &di)) != NVFP4_OK) return st;
+        size_t flags_off, partial_off;
+        const size_t base = workspace_layout(di->sms, &flags_off, &partial_off);
+        return nvfp4_tc::launch_dual(g_encode, di->sms, w_gate, s_gate, global_gate, w_up, s_up,
+                                     global_up, x, ldx, y, ldy, m, n, k, workspace,
+                                     workspace_bytes, base, stream);
+    }
     const uint8_t* ws_[2] = {w_gate, w_up};
     const uint8_t* ss_[2] = {s_gate, s_up};
     const float gs[2] = {global_gate, global_up};

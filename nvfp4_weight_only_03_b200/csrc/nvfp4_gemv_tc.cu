@@ -68,8 +68,9 @@ constexpr size_t smem_bytes(int nx) {
 constexpr size_t kSmemMax = smem_bytes(kMaxXRows);
 
 struct TcParams {
-    uint16_t* y;        // bf16 [M][ldy] (written when splits == 1)
+    uint16_t* y;        // bf16 [M][ldy] (written when splits == 1 and yf is null)
     int64_t ldy;
+    float* yf;          // or fp32 [M][n], without g (the dual's two streams)
     int64_t n, k;
     int m;
     int nx;             // MMA N: M rounded up to 16
@@ -346,7 +347,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
                     if (n < p.n) {
                         const int cols = p.m - c0 < 32 ? p.m - c0 : 32;
-                        if (p.splits == 1) {
+                        if (p.splits == 1 && p.yf) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (j < cols)
+                                    p.yf[(int64_t)(c0 + j) * p.n + n] =
+                                        __uint_as_float(v[j]) * p.descale[c0 + j];
+                        } else if (p.splits == 1) {
 #pragma unroll
                             for (int j = 0; j < 32; ++j)
                                 if (j < cols)
@@ -371,9 +378,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                      "r"(kTmemCols));
 }
 
-// y[m][n] = bf16(g * 2^-e(m) * sum over splits, in split order, of the partials)
+// y[m][n] = bf16(g * 2^-e(m) * sum over splits, in split order, of the partials), or into yf
+// the fp32 2^-e(m) * sum
 __global__ void nvfp4_tc_reduce(const float* __restrict__ partial, const float* __restrict__ descale,
-                                uint16_t* y, int64_t ldy, int64_t n, int m, float g, int splits) {
+                                uint16_t* y, int64_t ldy, float* yf, int64_t n, int m, float g,
+                                int splits) {
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t total = (int64_t)m * n;
     if (idx >= total) return;
@@ -383,7 +392,19 @@ __global__ void nvfp4_tc_reduce(const float* __restrict__ partial, const float* 
     float acc = 0.f;
     for (int s = 0; s < splits; ++s)
         acc += partial[(((tile * splits + s) * (int64_t)m) + mm) * kRows + r];
-    y[(int64_t)mm * ldy + nn] = f2bf(acc * descale[mm] * g);
+    if (yf) yf[(int64_t)mm * n + nn] = acc * descale[mm];
+    else y[(int64_t)mm * ldy + nn] = f2bf(acc * descale[mm] * g);
+}
+
+// o[m][n] = bf16(silu(g_g gate) * (g_u up)), silu(t) = t / (1 + e^-t), in fp32
+__global__ void nvfp4_tc_silu_mul(const float* __restrict__ gate, const float* __restrict__ up,
+                                  uint16_t* y, int64_t ldy, int64_t n, int m, float gg, float gu) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)m * n) return;
+    const int mm = (int)(idx / n);
+    const int64_t nn = idx - (int64_t)mm * n;
+    const float a = gate[idx] * gg, b = up[idx] * gu;
+    y[(int64_t)mm * ldy + nn] = f2bf(a / (1.0f + expf(-a)) * b);
 }
 
 // The f16 copy of x: row m scaled by 2^e(m) so that its largest magnitude lands in
@@ -466,22 +487,36 @@ int choose_splits(int64_t n, int64_t k, int sms) {
 
 static size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
-// scratch of a call: fp32 partials (when K is split), the f16 copy of x, the row descales
-size_t scratch_bytes(int64_t n, int64_t k, int m, int sms) {
+// Scratch of a call: fp32 partials (when K is split), the f16 copy of x, the row descales, and
+// for the dual the two streams' fp32 results.
+struct Scratch {
+    size_t partial, x16, descale, gate, up, total;
+};
+
+static Scratch scratch_layout(int64_t n, int64_t k, int m, int sms, bool dual) {
     const int64_t tiles = (n + kRows - 1) / kRows;
     const int splits = choose_splits(n, k, sms);
+    Scratch sc;
+    sc.partial = 0;
     const size_t partial = splits > 1 ? (size_t)tiles * splits * m * kRows * sizeof(float) : 0;
-    return align256(partial) + align256((size_t)m * k * 2) + align256((size_t)m * sizeof(float));
+    sc.x16 = align256(partial);
+    sc.descale = sc.x16 + align256((size_t)m * k * 2);
+    sc.gate = sc.descale + align256((size_t)m * sizeof(float));
+    const size_t res = dual ? align256((size_t)m * n * sizeof(float)) : 0;
+    sc.up = sc.gate + res;
+    sc.total = sc.up + res;
+    return sc;
+}
+
+size_t scratch_bytes(int64_t n, int64_t k, int m, int sms) {
+    return scratch_layout(n, k, m, sms, true).total;  // covers the single and the dual
 }
 
 bool usable(const void* s, int64_t k) {
     return (k % kUnitK) == 0 && (reinterpret_cast<uintptr_t>(s) & 15u) == 0;
 }
 
-int launch(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g, const void* x,
-           int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws,
-           size_t ws_bytes, size_t scratch_off, cudaStream_t stream) {
-    if (ws_bytes < scratch_off + scratch_bytes(n, k, m, sms)) return NVFP4_ERR_WORKSPACE;
+static int set_attr() {
     static bool attr_set[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
@@ -496,26 +531,29 @@ int launch(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g
         }
         attr_set[dev] = true;
     }
+    return NVFP4_OK;
+}
+
+// The weight's tile pass over the f16 copy of x (already written), then the split reduction.
+static int enqueue_weight(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g,
+                          const uint16_t* x16, const float* descale, float* partial, int m, int64_t n,
+                          int64_t k, uint16_t* y, int64_t ldy, float* yf, int32_t* error,
+                          cudaStream_t stream) {
+    const int tiles = (int)((n + kRows - 1) / kRows);
+    const int splits = choose_splits(n, k, sms);
+    const int nx = (m + 15) / 16 * 16;  // MMA N
     CUtensorMap tx, tw, ts;
     memset(&tx, 0, sizeof(tx));
     memset(&tw, 0, sizeof(tw));
     memset(&ts, 0, sizeof(ts));
-    const int tiles = (int)((n + kRows - 1) / kRows);
-    const int splits = choose_splits(n, k, sms);
-    const int nx = (m + 15) / 16 * 16;  // MMA N
-    char* const scratch = static_cast<char*>(ws) + scratch_off;
-    const size_t partial = splits > 1 ? (size_t)tiles * splits * m * kRows * sizeof(float) : 0;
-    uint16_t* const x16 = reinterpret_cast<uint16_t*>(scratch + align256(partial));
-    float* const descale =
-        reinterpret_cast<float*>(scratch + align256(partial) + align256((size_t)m * k * 2));
     const cuuint32_t one[2] = {1, 1};
     {
         // the f16 copy of x: [M][K], box 64 k x N rows, 128-byte swizzle; rows >= M read as zero
         const cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)m};
         const cuuint64_t strides[1] = {(cuuint64_t)k * 2};
         const cuuint32_t box[2] = {(cuuint32_t)kStageK, (cuuint32_t)nx};
-        if (encode(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, dims, strides, box, one,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+        if (encode(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(x16), dims,
+                   strides, box, one, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
             CUDA_SUCCESS)
             return NVFP4_ERR_LAUNCH;
@@ -542,8 +580,9 @@ int launch(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g
     }
     TcParams p;
     memset(&p, 0, sizeof(p));
-    p.y = static_cast<uint16_t*>(y);
+    p.y = y;
     p.ldy = ldy;
+    p.yf = yf;
     p.n = n;
     p.k = k;
     p.m = m;
@@ -554,20 +593,64 @@ int launch(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g
     p.tiles = tiles;
     p.splits = splits;
     p.units = (int)((k + kUnitK - 1) / kUnitK);
-    p.error = static_cast<int32_t*>(ws);
-    p.partial = reinterpret_cast<float*>(scratch);
-    nvfp4_tc_prep<<<m, 512, 0, stream>>>(static_cast<const uint16_t*>(x), ldx, k, x16, descale);
-    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
-    const size_t smem = smem_bytes(nx);
-    nvfp4_tc_kernel<<<tiles * splits, kThreads, smem, stream>>>(p, tx, tw, ts);
+    p.error = error;
+    p.partial = partial;
+    nvfp4_tc_kernel<<<tiles * splits, kThreads, smem_bytes(nx), stream>>>(p, tx, tw, ts);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
     if (splits > 1) {
         const int64_t total = (int64_t)m * n;
         const int threads = 256;
         nvfp4_tc_reduce<<<(unsigned)((total + threads - 1) / threads), threads, 0, stream>>>(
-            p.partial, descale, p.y, ldy, n, m, g, splits);
+            partial, descale, y, ldy, yf, n, m, g, splits);
         if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
     }
+    return NVFP4_OK;
+}
+
+int launch(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g, const void* x,
+           int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws,
+           size_t ws_bytes, size_t scratch_off, cudaStream_t stream) {
+    if (ws_bytes < scratch_off + scratch_bytes(n, k, m, sms)) return NVFP4_ERR_WORKSPACE;
+    int st = set_attr();
+    if (st != NVFP4_OK) return st;
+    const Scratch sc = scratch_layout(n, k, m, sms, false);
+    char* const base = static_cast<char*>(ws) + scratch_off;
+    uint16_t* const x16 = reinterpret_cast<uint16_t*>(base + sc.x16);
+    float* const descale = reinterpret_cast<float*>(base + sc.descale);
+    nvfp4_tc_prep<<<m, 512, 0, stream>>>(static_cast<const uint16_t*>(x), ldx, k, x16, descale);
+    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
+    return enqueue_weight(encode, sms, w, s, g, x16, descale,
+                          reinterpret_cast<float*>(base + sc.partial), m, n, k,
+                          static_cast<uint16_t*>(y), ldy, nullptr, static_cast<int32_t*>(ws), stream);
+}
+
+int launch_dual(EncodeFn encode, int sms, const uint8_t* wg, const uint8_t* sg, float gg,
+                const uint8_t* wu, const uint8_t* su, float gu, const void* x, int64_t ldx,
+                void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws, size_t ws_bytes,
+                size_t scratch_off, cudaStream_t stream) {
+    if (ws_bytes < scratch_off + scratch_bytes(n, k, m, sms)) return NVFP4_ERR_WORKSPACE;
+    int st = set_attr();
+    if (st != NVFP4_OK) return st;
+    const Scratch sc = scratch_layout(n, k, m, sms, true);
+    char* const base = static_cast<char*>(ws) + scratch_off;
+    uint16_t* const x16 = reinterpret_cast<uint16_t*>(base + sc.x16);
+    float* const descale = reinterpret_cast<float*>(base + sc.descale);
+    float* const partial = reinterpret_cast<float*>(base + sc.partial);
+    float* const gate = reinterpret_cast<float*>(base + sc.gate);
+    float* const up = reinterpret_cast<float*>(base + sc.up);
+    int32_t* const error = static_cast<int32_t*>(ws);
+    nvfp4_tc_prep<<<m, 512, 0, stream>>>(static_cast<const uint16_t*>(x), ldx, k, x16, descale);
+    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
+    if ((st = enqueue_weight(encode, sms, wg, sg, gg, x16, descale, partial, m, n, k, nullptr, 0,
+                             gate, error, stream)) != NVFP4_OK)
+        return st;
+    if ((st = enqueue_weight(encode, sms, wu, su, gu, x16, descale, partial, m, n, k, nullptr, 0,
+                             up, error, stream)) != NVFP4_OK)
+        return st;
+    const int64_t total = (int64_t)m * n;
+    nvfp4_tc_silu_mul<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(
+        gate, up, static_cast<uint16_t*>(y), ldy, n, m, gg, gu);
+    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
     return NVFP4_OK;
 }
 

@@ -16,8 +16,8 @@ using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, voi
 
 // K-splits of an N x K call (depends only on N, K and the SM count).
 int choose_splits(int64_t n, int64_t k, int sms);
-// Scratch bytes of a tier call of m rows: fp32 partials (when K is split), an f16 copy of x and
-// the rows' scales.
+// Scratch bytes of a tier call of m rows (single or dual): fp32 partials (when K is split), an
+// f16 copy of x, the rows' scales, and the dual's two fp32 results.
 size_t scratch_bytes(int64_t n, int64_t k, int m, int sms);
 // The tier's TMA scale boxes need K % 256 == 0 and 16-byte aligned scale codes.
 bool usable(const void* s, int64_t k);
@@ -26,6 +26,12 @@ bool usable(const void* s, int64_t k);
 int launch(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g, const void* x,
            int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws,
            size_t ws_bytes, size_t scratch_off, cudaStream_t stream);
+// The fused dual: o = bf16(silu(g_g W_gate x) * (g_u W_up x)), the two streams through the tier
+// into fp32, then one combining pass.
+int launch_dual(EncodeFn encode, int sms, const uint8_t* wg, const uint8_t* sg, float gg,
+                const uint8_t* wu, const uint8_t* su, float gu, const void* x, int64_t ldx,
+                void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws, size_t ws_bytes,
+                size_t scratch_off, cudaStream_t stream);
 
 }  // namespace nvfp4_tc
 

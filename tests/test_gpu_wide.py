@@ -1,7 +1,8 @@
 """The tensor-core tier for 9..128 rows (NVFP4_FLAG_WIDE_TENSOR) through the C ABI against the
 fp64 oracle under the acceptance rules; bitwise row invariance over M = 9..128 and determinism;
-both ways of finishing a tile (direct, or fp32 partials of a K split added in order); and the
-fall-back to 8-row passes where the tier does not apply."""
+both ways of finishing a tile (direct, or fp32 partials of a K split added in order); the fused
+dual (gate and up through the tier in fp32, then SiLU(gate)*up); and the fall-back to 8-row
+passes where the tier does not apply."""
 import numpy as np
 import pytest
 import torch
@@ -9,7 +10,7 @@ import torch
 import oracle
 import synth
 import nvfp4_weight_only_03_b200 as nv
-from gpu_util import bits, check_single, dev_weight, dev_x
+from gpu_util import bits, check_dual, check_single, dev_weight, dev_x
 
 pytestmark = pytest.mark.gpu
 
@@ -89,3 +90,64 @@ def test_tier_rejects_a_small_workspace():
     with pytest.raises(nv.Nvfp4Error) as e:
         nv.gemv(W, S, 1.0, x, ws=ws, wide_tensor=True)
     assert e.value.status == -7
+
+
+def wide_dual(Wg, Sg, gg, Wu, Su, gu, x_dev):
+    o = nv.gemv_dual(Wg, Sg, gg, Wu, Su, gu, x_dev, wide_tensor=True)
+    torch.cuda.synchronize()
+    return bits(o)
+
+
+@pytest.mark.parametrize("n,k,m", [
+    (2048, 5120, 24),        # K split: both streams reduced into fp32 before the combine
+    (1000 + 77, 1024, 40),   # ragged N
+    (148 * 128, 512, 128),   # no K split: the tier writes the fp32 results itself
+])
+def test_dual_tier_matches_oracle(n, k, m):
+    wg = synth.nvfp4_weight(34, 0, n, k)
+    wu = synth.nvfp4_weight(34, 40_000_000, n, k)
+    x = synth.activations(34, 80_000_000, m, k)
+    Wg, Sg, gg = dev_weight(wg)
+    Wu, Su, gu = dev_weight(wu)
+    o = wide_dual(Wg, Sg, gg, Wu, Su, gu, dev_x(x))
+    rows = None if n <= 2048 else np.unique(
+        np.concatenate([np.random.default_rng(n).integers(0, n, 150), [0, 127, 128, n - 1]]))
+    o_ref, yg, yu, ag, au = oracle.gemv_dual(wg.packed, wg.scales, wg.g, wu.packed, wu.scales,
+                                             wu.g, x, rows=rows)
+    check_dual(o if rows is None else o[:, rows], o_ref, yg, yu, ag, au,
+               f"dual tier n={n} k={k} M={m}")
+    assert nv.workspace_error(nv.wide_workspace(n, k, m)) == 0
+
+
+def test_dual_tier_rows_invariant_and_deterministic():
+    n, k = 2048, 5120
+    wg = synth.nvfp4_weight(35, 0, n, k)
+    wu = synth.nvfp4_weight(35, 20_000_000, n, k)
+    x = synth.activations(35, 40_000_000, 128, k)
+    Wg, Sg, gg = dev_weight(wg)
+    Wu, Su, gu = dev_weight(wu)
+    o128 = wide_dual(Wg, Sg, gg, Wu, Su, gu, dev_x(x))
+    for m in (9, 64):
+        assert np.array_equal(wide_dual(Wg, Sg, gg, Wu, Su, gu, dev_x(x[:m])), o128[:m]), m
+    assert np.array_equal(wide_dual(Wg, Sg, gg, Wu, Su, gu, dev_x(x[30:47])), o128[30:47])
+    assert np.array_equal(wide_dual(Wg, Sg, gg, Wu, Su, gu, dev_x(x)), o128)
+
+
+def test_dual_tier_strided_and_fallback():
+    n, k, m = 900, 2048, 20
+    wg = synth.nvfp4_weight(36, 0, n, k)
+    wu = synth.nvfp4_weight(36, 4_000_000, n, k)
+    x = synth.activations(36, 8_000_000, m, k)
+    Wg, Sg, gg = dev_weight(wg)
+    Wu, Su, gu = dev_weight(wu)
+    ybuf = torch.full((m, n + 24), float("nan"), dtype=torch.bfloat16, device="cuda")
+    o = nv.gemv_dual(Wg, Sg, gg, Wu, Su, gu, dev_x(x, ldx=k + 128), y=ybuf[:, :n],
+                     wide_tensor=True)
+    torch.cuda.synchronize()
+    o_ref, yg, yu, ag, au = oracle.gemv_dual(wg.packed, wg.scales, wg.g, wu.packed, wu.scales,
+                                             wu.g, x)
+    check_dual(bits(o), o_ref, yg, yu, ag, au, "dual tier strided")
+    assert torch.isnan(ybuf[:, n:].float()).all()
+    # 1..8 rows ignore the flag (bitwise the fused dual kernel)
+    o8 = wide_dual(Wg, Sg, gg, Wu, Su, gu, dev_x(x[:8]))
+    assert np.array_equal(o8, bits(nv.gemv_dual(Wg, Sg, gg, Wu, Su, gu, dev_x(x[:8]))))
