@@ -13,6 +13,11 @@ Parity status of each function (what pins it is listed in the tests named here):
   gemv ..................... pinned: closed-form sums, brute force, invariants, library matmul
                              cross-check (tests/test_oracle_gemv.py)
   gemv_dual ................ pinned: SiLU closed forms + reduction to gemv (tests/test_oracle_gemv.py)
+  add_rmsnorm .............. pinned: hand-derived values, closed forms of the mean square and eps,
+                             tie rounding of the residual sum, scale and sign invariants, a
+                             50-digit decimal brute force (tests/test_oracle_prologue.py)
+  sigmoid_gate ............. pinned: sigmoid(0) = 1/2, saturation, the symmetry
+                             sigmoid(t) + sigmoid(-t) = 1, decimal brute force (same file)
 """
 from __future__ import annotations
 
@@ -58,6 +63,11 @@ def _load():
         lib.oracle_gemv_dual.argtypes = [vp, vp, ctypes.c_float, vp, vp, ctypes.c_float, vp, i64,
                                          c_int, i64, i64, vp, i64, vp, vp, vp, vp, vp, c_int]
         lib.oracle_gemv_dual.restype = c_int
+        lib.oracle_add_rmsnorm.argtypes = [vp, i64, vp, i64, vp, ctypes.c_float, c_int, i64, vp,
+                                           vp, vp]
+        lib.oracle_add_rmsnorm.restype = c_int
+        lib.oracle_sigmoid_gate.argtypes = [vp, i64, vp, i64, c_int, i64, vp, vp]
+        lib.oracle_sigmoid_gate.restype = c_int
         _lib = lib
     return _lib
 
@@ -149,6 +159,61 @@ def gemv_dual(pg, sg, gg, pu, su, gu, x, rows=None, threads: int = 0):
     if rc:
         raise ValueError("oracle_gemv_dual rejected its arguments")
     return tuple(outs)
+
+
+def add_rmsnorm(x, r, gamma, eps: float):
+    """Residual add, then RMS norm with gain (x, r: bf16 bits [m][k]; gamma: bf16 bits [k]).
+    Returns (h, xn, near): h = bf16(x + r), xn = bf16(h * gamma / sqrt(mean(h^2) + eps)), both
+    bf16 bits [m][k], and near[m][k] = 1 where xn's fp64 value lies within a relative 2^-16 of a
+    bf16 rounding midpoint."""
+    x, px = _c(np.atleast_2d(x), np.uint16)
+    r, pr = _c(np.atleast_2d(r), np.uint16)
+    gamma, pg = _c(gamma, np.uint16)
+    m, k = x.shape
+    if r.shape != (m, k) or gamma.shape != (k,):
+        raise ValueError("x and r must be [m][k], gamma [k]")
+    h = np.zeros((m, k), np.uint16)
+    xn = np.zeros((m, k), np.uint16)
+    near = np.zeros((m, k), np.uint8)
+    rc = _load().oracle_add_rmsnorm(px, k, pr, k, pg, eps, m, k, h.ctypes.data, xn.ctypes.data,
+                                    near.ctypes.data)
+    if rc:
+        raise ValueError("oracle_add_rmsnorm rejected its arguments")
+    return h, xn, near
+
+
+def sigmoid_gate(a, gate):
+    """xo = bf16(a * sigmoid(gate)) (bf16 bits [m][k] in and out) and its near-midpoint mask."""
+    a, pa = _c(np.atleast_2d(a), np.uint16)
+    gate, pg = _c(np.atleast_2d(gate), np.uint16)
+    m, k = a.shape
+    if gate.shape != (m, k):
+        raise ValueError("a and gate must be [m][k]")
+    xo = np.zeros((m, k), np.uint16)
+    near = np.zeros((m, k), np.uint8)
+    rc = _load().oracle_sigmoid_gate(pa, k, pg, k, m, k, xo.ctypes.data, near.ctypes.data)
+    if rc:
+        raise ValueError("oracle_sigmoid_gate rejected its arguments")
+    return xo, near
+
+
+def rounding_slack(xq, near) -> np.ndarray:
+    """bf16 bits [m][k]: the larger gap from each near-midpoint element of xq to a bf16
+    neighbour (a power of two), zero elsewhere.  The GEMV of these (its absolute-sum output)
+    bounds how far y moves when those elements round the other way."""
+    xq = np.asarray(xq, np.uint16)
+    o = bf16_ordinal(xq)
+
+    def from_ordinal(v):
+        v = np.asarray(v, np.int64)
+        mag = np.abs(v).astype(np.uint16)
+        return np.where(v < 0, mag | 0x8000, mag).astype(np.uint16)
+
+    v = bf16_value(xq)
+    gap = np.maximum(np.abs(bf16_value(from_ordinal(o + 1)) - v),
+                     np.abs(v - bf16_value(from_ordinal(o - 1))))
+    gap = np.where(np.asarray(near) != 0, gap, 0.0)
+    return bf16_rne(gap)
 
 
 # ----------------------------------------------------------------------------------------------

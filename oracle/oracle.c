@@ -22,6 +22,14 @@
  * all in fp64 (the SiLU(gate)*up of the SwiGLU FFN that the GB10 plan runs as
  * w4a16_gemv_dual_sw followed by moe_silu_mul).
  *
+ * Input prologues (the GEMV's neighbours in the decode step: "residual_add_rms_norm",
+ * "rms_norm" and "sigmoid_gate_mul" in the same page's table "Kernels the plan launches"; the
+ * pages list them by name, the formulas are the standard RMS normalisation with a gain and
+ * the sigmoid output gate of gated attention):
+ *   add + RMS norm:  h = bf16(x + r);  xn = bf16(h * gamma / sqrt(mean_k(h^2) + eps))
+ *   sigmoid gate:    xo = bf16(a * sigmoid(gate)),  sigmoid(t) = 1 / (1 + exp(-t))
+ * in fp64 with one rounding to bf16 at the end of each line.
+ *
  * Formats, written from their definitions (the pages name the format, not its bits):
  *   E2M1 nibble: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0;
  *                exponent 0 is subnormal: 0.5 * m.
@@ -146,5 +154,73 @@ int oracle_gemv_dual(const uint8_t* wg, const uint8_t* sg, float gg, const uint8
         double t = yg[i];
         o[i] = t / (1.0 + exp(-t)) * yu[i];
     }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------------------- */
+/* input prologues */
+
+/* bf16 neighbours by ordinal (finite values; +0 and -0 share ordinal 0) */
+static double bf16_step(uint16_t b, int dir) {
+    int32_t o = (b & 0x8000) ? -(int32_t)(b & 0x7FFF) : (int32_t)(b & 0x7FFF);
+    o += dir;
+    uint16_t n = o < 0 ? (uint16_t)(0x8000 | (uint16_t)(-o)) : (uint16_t)o;
+    return oracle_bf16_value(n);
+}
+
+/* 1 when v lies within a relative 2^-16 of a midpoint between bf16 neighbours, i.e. where an
+ * evaluation less precise than fp64 may round the other way; 0 otherwise. */
+static uint8_t near_midpoint(double v, uint16_t b) {
+    if (v == 0.0 || (b & 0x7FFF) >= 0x7F80) return 0;
+    double c = oracle_bf16_value(b);
+    double lo = 0.5 * (c + bf16_step(b, -1)), hi = 0.5 * (c + bf16_step(b, +1));
+    double d = fmin(fabs(v - lo), fabs(v - hi));
+    return d <= ldexp(fabs(v), -16) ? 1 : 0;
+}
+
+/* Residual add, then RMS normalisation with a gain, row by row:
+ *   h[m][k]  = bf16_rne(x[m][k] + r[m][k])     (the exact sum of two bf16 values, rounded once)
+ *   ms[m]    = (1/K) sum_k h[m][k]^2           (fp64, increasing k)
+ *   xn[m][k] = bf16_rne(h[m][k] * gamma[k] / sqrt(ms[m] + eps))
+ * h is [m][k] (row stride k), xn likewise; near (may be NULL) marks xn elements whose fp64
+ * value lies within a relative 2^-16 of a bf16 rounding midpoint. */
+int oracle_add_rmsnorm(const uint16_t* x, int64_t ldx, const uint16_t* r, int64_t ldr,
+                       const uint16_t* gamma, float eps, int m, int64_t k, uint16_t* h,
+                       uint16_t* xn, uint8_t* near) {
+    if (m < 0 || k <= 0 || ldx < k || ldr < k || !x || !r || !gamma || !h || !xn) return -1;
+    if (!(eps >= 0.0f) || isinf(eps)) return -1;
+    for (int i = 0; i < m; ++i) {
+        double ss = 0.0;
+        for (int64_t j = 0; j < k; ++j) {
+            uint16_t hb = oracle_bf16_rne(oracle_bf16_value(x[i * ldx + j]) +
+                                          oracle_bf16_value(r[i * ldr + j]));
+            h[i * k + j] = hb;
+            double hv = oracle_bf16_value(hb);
+            ss += hv * hv;
+        }
+        double inv = 1.0 / sqrt(ss / (double)k + (double)eps);
+        for (int64_t j = 0; j < k; ++j) {
+            double v = oracle_bf16_value(h[i * k + j]) * oracle_bf16_value(gamma[j]) * inv;
+            uint16_t b = oracle_bf16_rne(v);
+            xn[i * k + j] = b;
+            if (near) near[i * k + j] = near_midpoint(v, b);
+        }
+    }
+    return 0;
+}
+
+/* xo[m][k] = bf16_rne(a[m][k] * sigmoid(gate[m][k])), sigmoid(t) = 1 / (1 + exp(-t)) in fp64;
+ * xo is [m][k]; near as above. */
+int oracle_sigmoid_gate(const uint16_t* a, int64_t lda, const uint16_t* gate, int64_t ldg, int m,
+                        int64_t k, uint16_t* xo, uint8_t* near) {
+    if (m < 0 || k <= 0 || lda < k || ldg < k || !a || !gate || !xo) return -1;
+    for (int i = 0; i < m; ++i)
+        for (int64_t j = 0; j < k; ++j) {
+            double t = oracle_bf16_value(gate[i * ldg + j]);
+            double v = oracle_bf16_value(a[i * lda + j]) * (1.0 / (1.0 + exp(-t)));
+            uint16_t b = oracle_bf16_rne(v);
+            xo[i * k + j] = b;
+            if (near) near[i * k + j] = near_midpoint(v, b);
+        }
     return 0;
 }
