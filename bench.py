@@ -52,7 +52,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("sweep", "attn_pairs", "wide_rows"), default="sweep")
+    ap.add_argument("--workload", choices=("sweep", "attn_pairs", "wide_rows", "prologue_layers"),
+                    default="sweep")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -809,6 +810,343 @@ def run_pairs(args, world, rank, local):
 
 
 # ----------------------------------------------------------------------------------------------
+# input prologues: the decode layer's neighbours of the GEMV fused into its x staging
+
+PRO_ROWS = (1, 8)
+PRO_EPS = 1e-6
+PRO_DESC = ("decode-step sweep (4 layers x {qkv 10240x5120, o 5120x6144, gate_up dual 2x17408x5120, "
+            "down 5120x17408} NVFP4, M in {1,8}) with the layer's neighbours fused as input "
+            "prologues: residual add + RMS norm before qkv and gate_up (h written out), the sigmoid "
+            "gate before o; x of each layer is the previous down output. Also timed: the same "
+            "GEMVs without the neighbours, and with them as separate torch eager kernels")
+
+
+def prologue_step_bytes(wl, rows=PRO_ROWS):
+    """Algorithmic bytes of one step: every weight and scale once per M pass, x and y of each
+    call, and the prologue's operands (residual, gamma and h for the norm, the gate)."""
+    b = 0
+    for m in rows:
+        for p in wl.projections:
+            b += (2 if p.dual else 1) * (p.n * p.k // 2 + p.n * p.k // 16)
+            b += m * p.k * 2 + m * p.n * 2
+            kind = p.name.split(".")[1]
+            if kind in ("qkv", "gate_up"):
+                b += 2 * m * p.k * 2 + p.k * 2   # residual in, h out, gamma
+            elif kind == "o":
+                b += m * p.k * 2                 # gate
+    return b
+
+
+def run_prologue(args, world, rank, local):
+    import torch
+    import nvfp4_weight_only_03_b200 as nv
+    L = nv.lib()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = synth.make(WORKLOAD, generate_x=False)
+    seed = wl.seed
+    k_model = wl.projections[0].k          # 5120, the hidden size
+    k_attn = [p for p in wl.projections if p.name.endswith(".o")][0].k  # 6144
+
+    def bf16(bits_):
+        return torch.from_numpy(np.ascontiguousarray(bits_).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    ents = []
+    for p in wl.projections:
+        e = {"p": p, "W": torch.from_numpy(p.w.packed).to(dev),
+             "S": torch.from_numpy(p.w.scales).to(dev), "g": p.w.g,
+             "y": torch.empty((8, p.n), dtype=torch.bfloat16, device=dev)}
+        if p.dual:
+            e["Wu"] = torch.from_numpy(p.w_up.packed).to(dev)
+            e["Su"] = torch.from_numpy(p.w_up.scales).to(dev)
+            e["gu"] = p.w_up.g
+        ents.append(e)
+    # activations: the first layer's input and residual, the attention output and its gate per
+    # layer, one gain vector per norm; qkv's norm writes h to hbuf[0], gate_up's reads it and
+    # writes hbuf[1], the next layer's residual
+    x0 = bf16(synth.activations(seed + 200, 0, 8, k_model))
+    r0 = bf16(synth.residual_stream(seed + 200, 2 * 8 * k_model, 8, k_model))
+    n_layers = len(ents) // 4
+    attn = [bf16(synth.activations(seed + 201 + i, 0, 8, k_attn)) for i in range(n_layers)]
+    gates = [bf16(synth.gate_logits(seed + 201 + i, 2 * 8 * k_attn, 8, k_attn))
+             for i in range(n_layers)]
+    gammas = [bf16(synth.norm_gains(seed + 210 + i, 0, k_model)) for i in range(2 * n_layers)]
+    hbuf = [torch.empty((8, k_model), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    ws = nv.wide_workspace(k_attn, k_attn, 8, dev)  # holds the prologue's x' of 8 rows
+    wsp, wsn = ws.data_ptr(), ws.numel()
+    flags = nv.FLAG_PREFETCH_WEIGHTS
+    step_bytes_ = prologue_step_bytes(wl)
+
+    def plan(h):
+        """[(fn, args, keepalive)] for one fused step: per M, per layer qkv, o, gate_up, down."""
+        seq = []
+        for m in PRO_ROWS:
+            x, r = x0, r0
+            for li in range(n_layers):
+                qkv, o, gu, down = ents[4 * li:4 * li + 4]
+                # qkv: x' = rmsnorm(x + r), h -> hbuf[0]
+                pq = nv.Prologue(kind=nv.PROLOGUE_ADD_RMSNORM, eps=PRO_EPS, residual=r.data_ptr(),
+                                 ld_residual=k_model, gamma=gammas[2 * li].data_ptr(),
+                                 residual_out=hbuf[0].data_ptr(), ld_residual_out=k_model)
+                seq.append((L.nvfp4_gemv_pro, (ctypes.byref(pq), qkv["W"].data_ptr(),
+                            qkv["S"].data_ptr(), ctypes.c_float(qkv["g"]), x.data_ptr(), k_model,
+                            qkv["y"].data_ptr(), qkv["p"].n, m, qkv["p"].n, k_model, wsp, wsn,
+                            flags, h), pq))
+                # o: x' = attention output * sigmoid(gate)
+                po = nv.Prologue(kind=nv.PROLOGUE_SIGMOID_GATE, gate=gates[li].data_ptr(),
+                                 ld_gate=k_attn)
+                seq.append((L.nvfp4_gemv_pro, (ctypes.byref(po), o["W"].data_ptr(),
+                            o["S"].data_ptr(), ctypes.c_float(o["g"]), attn[li].data_ptr(),
+                            k_attn, o["y"].data_ptr(), o["p"].n, m, o["p"].n, k_attn, wsp, wsn,
+                            flags, h), po))
+                # gate_up: x' = rmsnorm(o + h), the new h -> hbuf[1]
+                pg = nv.Prologue(kind=nv.PROLOGUE_ADD_RMSNORM, eps=PRO_EPS,
+                                 residual=hbuf[0].data_ptr(), ld_residual=k_model,
+                                 gamma=gammas[2 * li + 1].data_ptr(),
+                                 residual_out=hbuf[1].data_ptr(), ld_residual_out=k_model)
+                seq.append((L.nvfp4_gemv_dual_pro, (ctypes.byref(pg), gu["W"].data_ptr(),
+                            gu["S"].data_ptr(), ctypes.c_float(gu["g"]), gu["Wu"].data_ptr(),
+                            gu["Su"].data_ptr(), ctypes.c_float(gu["gu"]), o["y"].data_ptr(),
+                            k_model, gu["y"].data_ptr(), gu["p"].n, m, gu["p"].n, k_model, wsp,
+                            wsn, flags, h), pg))
+                seq.append((L.nvfp4_gemv_ex, (down["W"].data_ptr(), down["S"].data_ptr(),
+                            ctypes.c_float(down["g"]), gu["y"].data_ptr(), down["p"].k,
+                            down["y"].data_ptr(), down["p"].n, m, down["p"].n, down["p"].k, wsp,
+                            wsn, flags, h), None))
+                x, r = down["y"], hbuf[1]
+        return seq
+
+    def plain(h):
+        """The same GEMVs on the same inputs without their neighbours."""
+        seq = []
+        for m in PRO_ROWS:
+            x = x0
+            for li in range(n_layers):
+                qkv, o, gu, down = ents[4 * li:4 * li + 4]
+                seq.append((L.nvfp4_gemv_ex, (qkv["W"].data_ptr(), qkv["S"].data_ptr(),
+                            ctypes.c_float(qkv["g"]), x.data_ptr(), k_model, qkv["y"].data_ptr(),
+                            qkv["p"].n, m, qkv["p"].n, k_model, wsp, wsn, flags, h), None))
+                seq.append((L.nvfp4_gemv_ex, (o["W"].data_ptr(), o["S"].data_ptr(),
+                            ctypes.c_float(o["g"]), attn[li].data_ptr(), k_attn,
+                            o["y"].data_ptr(), o["p"].n, m, o["p"].n, k_attn, wsp, wsn, flags,
+                            h), None))
+                seq.append((L.nvfp4_gemv_dual_ex, (gu["W"].data_ptr(), gu["S"].data_ptr(),
+                            ctypes.c_float(gu["g"]), gu["Wu"].data_ptr(), gu["Su"].data_ptr(),
+                            ctypes.c_float(gu["gu"]), o["y"].data_ptr(), k_model,
+                            gu["y"].data_ptr(), gu["p"].n, m, gu["p"].n, k_model, wsp, wsn,
+                            flags, h), None))
+                seq.append((L.nvfp4_gemv_ex, (down["W"].data_ptr(), down["S"].data_ptr(),
+                            ctypes.c_float(down["g"]), gu["y"].data_ptr(), down["p"].k,
+                            down["y"].data_ptr(), down["p"].n, m, down["p"].n, down["p"].k, wsp,
+                            wsn, flags, h), None))
+                x = down["y"]
+        return seq
+
+    stream = torch.cuda.Stream(device=dev)
+    xn_buf = torch.empty((8, k_model), dtype=torch.bfloat16, device=dev)
+    xg_buf = torch.empty((8, k_attn), dtype=torch.bfloat16, device=dev)
+
+    def torch_norm(x, r, gamma, hout, m):
+        h = (x[:m].float() + r[:m].float()).to(torch.bfloat16)
+        hout[:m].copy_(h)
+        hf = h.float()
+        xn = hf * torch.rsqrt(hf.pow(2).mean(-1, keepdim=True) + PRO_EPS) * gamma.float()
+        xn_buf[:m].copy_(xn.to(torch.bfloat16))
+
+    def run_separate(h):
+        """The neighbours as torch eager kernels, the GEMVs plain on their outputs."""
+        for m in PRO_ROWS:
+            x, r = x0, r0
+            for li in range(n_layers):
+                qkv, o, gu, down = ents[4 * li:4 * li + 4]
+                torch_norm(x, r, gammas[2 * li], hbuf[0], m)
+                fns = [(L.nvfp4_gemv_ex, (qkv["W"].data_ptr(), qkv["S"].data_ptr(),
+                        ctypes.c_float(qkv["g"]), xn_buf.data_ptr(), k_model, qkv["y"].data_ptr(),
+                        qkv["p"].n, m, qkv["p"].n, k_model, wsp, wsn, flags, h))]
+                for fn, a in fns:
+                    if fn(*a) != 0:
+                        raise RuntimeError("launch failed")
+                xg_buf[:m].copy_((attn[li][:m].float() * torch.sigmoid(gates[li][:m].float()))
+                                 .to(torch.bfloat16))
+                if L.nvfp4_gemv_ex(o["W"].data_ptr(), o["S"].data_ptr(), ctypes.c_float(o["g"]),
+                                   xg_buf.data_ptr(), k_attn, o["y"].data_ptr(), o["p"].n, m,
+                                   o["p"].n, k_attn, wsp, wsn, flags, h) != 0:
+                    raise RuntimeError("launch failed")
+                torch_norm(o["y"], hbuf[0], gammas[2 * li + 1], hbuf[1], m)
+                if L.nvfp4_gemv_dual_ex(gu["W"].data_ptr(), gu["S"].data_ptr(),
+                                        ctypes.c_float(gu["g"]), gu["Wu"].data_ptr(),
+                                        gu["Su"].data_ptr(), ctypes.c_float(gu["gu"]),
+                                        xn_buf.data_ptr(), k_model, gu["y"].data_ptr(), gu["p"].n,
+                                        m, gu["p"].n, k_model, wsp, wsn, flags, h) != 0:
+                    raise RuntimeError("launch failed")
+                if L.nvfp4_gemv_ex(down["W"].data_ptr(), down["S"].data_ptr(),
+                                   ctypes.c_float(down["g"]), gu["y"].data_ptr(), down["p"].k,
+                                   down["y"].data_ptr(), down["p"].n, m, down["p"].n,
+                                   down["p"].k, wsp, wsn, flags, h) != 0:
+                    raise RuntimeError("launch failed")
+                x, r = down["y"], hbuf[1]
+
+    def graph_of(build):
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 3)):
+                build(stream.cuda_stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            build(torch.cuda.current_stream().cuda_stream)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        return g
+
+    def run_seq(make):
+        def build(h):
+            for fn, a, _keep in make(h):
+                st = fn(*a)
+                if st != 0:
+                    raise RuntimeError(f"launch failed: {nv.STATUS.get(st, st)}")
+        return build
+
+    def timed(g, steps):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            t0.record()
+            for _ in range(steps):
+                g.replay()
+            t1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(t0.elapsed_time(t1), world)
+
+    n_launch = len(plan(0))
+    g_fused = graph_of(run_seq(plan))
+    g_plain = graph_of(run_seq(plain))
+    g_sep = graph_of(run_separate)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ms = timed(g_fused, args.steps)
+    clk = clocks.stop()
+    ms_plain = timed(g_plain, args.steps)
+    ms_sep = timed(g_sep, args.steps)
+    value = world * step_bytes_ * args.steps / (ms * 1e-3) / 1e9
+    peak, peak_src = peaks()
+    per_launch_us = ms / args.steps * 1e3 / n_launch
+    bytes_avg = step_bytes_ / n_launch
+
+    # end to end through the public API: the step's first input, residual, attention outputs and
+    # gates in from pinned host memory, the last down output of each M pass back
+    srcs = [x0, r0] + attn + gates
+    hx = torch.cat([t.reshape(-1) for t in srcs]).cpu().pin_memory()
+    dx = torch.empty_like(hx, device=dev)
+    views, off = [], 0
+    for t in srcs:
+        views.append(dx[off:off + t.numel()].view(t.shape))
+        off += t.numel()
+    ex0, er0 = views[0], views[1]
+    eattn, egates = views[2:2 + n_layers], views[2 + n_layers:]
+    last = ents[-1]
+    hy = torch.empty((len(PRO_ROWS), 8, last["p"].n), dtype=torch.bfloat16).pin_memory()
+    cur = torch.cuda.current_stream()
+
+    def e2e_step():
+        dx.copy_(hx, non_blocking=True)
+        for mi, m in enumerate(PRO_ROWS):
+            x, r = ex0[:m], er0[:m]
+            for li in range(n_layers):
+                qkv, o, gu, down = ents[4 * li:4 * li + 4]
+                nv.gemv(qkv["W"], qkv["S"], qkv["g"], x, y=qkv["y"][:m], ws=ws, stream=cur,
+                        prefetch_weights=True, prologue=nv.AddRmsNorm(
+                            r, gammas[2 * li], PRO_EPS, hbuf[0][:m]))
+                nv.gemv(o["W"], o["S"], o["g"], eattn[li][:m], y=o["y"][:m], ws=ws, stream=cur,
+                        prefetch_weights=True, prologue=nv.SigmoidGate(egates[li][:m]))
+                nv.gemv_dual(gu["W"], gu["S"], gu["g"], gu["Wu"], gu["Su"], gu["gu"], o["y"][:m],
+                             y=gu["y"][:m], ws=ws, stream=cur, prefetch_weights=True,
+                             prologue=nv.AddRmsNorm(hbuf[0][:m], gammas[2 * li + 1], PRO_EPS,
+                                                    hbuf[1][:m]))
+                nv.gemv(down["W"], down["S"], down["g"], gu["y"][:m], y=down["y"][:m], ws=ws,
+                        stream=cur, prefetch_weights=True)
+                x, r = down["y"][:m], hbuf[1][:m]
+            hy[mi, :m].copy_(last["y"][:m], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(cur)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    t1.record(cur)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(t0.elapsed_time(t1), world)
+    d2h = sum(m * last["p"].n * 2 for m in PRO_ROWS)
+    e2e = {"value": round(world * step_bytes_ * args.e2e_steps / (ms_e2e * 1e-3) / 1e9, 1),
+           "unit": "GB/s", "h2d_bytes_per_step": hx.numel() * 2, "d2h_bytes_per_step": d2h,
+           "steps": args.e2e_steps,
+           "api": "nvfp4_weight_only_03_b200.gemv / gemv_dual with AddRmsNorm / SigmoidGate"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        threads = os.cpu_count() or 1
+        xb = synth.activations(seed + 200, 0, 8, k_model)
+        rb = synth.residual_stream(seed + 200, 2 * 8 * k_model, 8, k_model)
+        gb = synth.norm_gains(seed + 210, 0, k_model)
+        qkv = wl.projections[0]
+        t_end = time.perf_counter() + args.cpu_seconds
+        b, n_calls, t_start = 0, 0, time.perf_counter()
+        while time.perf_counter() < t_end:
+            m = PRO_ROWS[n_calls % len(PRO_ROWS)]
+            _, xq, _ = oracle.add_rmsnorm(xb[:m], rb[:m], gb, PRO_EPS)
+            oracle.gemv(qkv.w.packed, qkv.w.scales, qkv.w.g, xq, rows=np.arange(256),
+                        threads=threads)
+            b += 256 * (qkv.k // 2 + qkv.k // 16) + 4 * m * qkv.k * 2 + qkv.k * 2 + m * 256 * 2
+            n_calls += 1
+        dt = time.perf_counter() - t_start
+        cpu = {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n_calls} calls of the norm prologue then 256 qkv output rows, M "
+                         f"alternating 1 and 8 ({dt:.1f} s)"}
+
+    del g_fused, g_plain, g_sep
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4(e2m1+e4m3) x bf16 -> fp32 accumulate, bf16 out",
+            "data": "synthetic (seeded N(0,0.02) weights quantised to NVFP4; N(0,1) x, N(0,16) "
+                    "residual, 1+N(0,0.01) gains, N(0,4) gate logits, all bf16)",
+            "config": {"workload": PRO_DESC, "rows": list(PRO_ROWS), "eps": PRO_EPS,
+                       "bytes_per_step": step_bytes_,
+                       "l2": "0.79 GB of weights per M pass > 126 MB L2; no flush",
+                       "launch": f"one CUDA graph per step ({n_launch} kernels, programmatic "
+                                 "dependent launch), persistent grid = SMs",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "kernel": "nvfp4_gemv_kernel (all instances)",
+                         "achieved": round(bytes_avg / (per_launch_us * 1e-6) / 1e9, 1),
+                         "peak": peak, "unit": "GB/s",
+                         "frac": round(bytes_avg / (per_launch_us * 1e-6) / 1e9 / peak, 4),
+                         "traffic": None, "peak_source": peak_src,
+                         "bytes_per_launch_avg": round(bytes_avg),
+                         "avg_launch_us": round(per_launch_us, 3),
+                         "timing": "CUDA events around the K timed steps; every launch of the "
+                                   "step is a GEMV kernel"},
+            "without_neighbours": {"ms_per_step": round(ms_plain / args.steps, 5),
+                                   "what": "the same GEMVs with no prologue (the neighbours' work "
+                                           "left out): the floor the fusion is measured against"},
+            "separate_torch_neighbours": {"ms_per_step": round(ms_sep / args.steps, 5),
+                                          "what": "plain GEMVs with the neighbours as torch "
+                                                  "eager kernels in the same graph"},
+            "e2e": e2e, "gpu_launches": n_launch * args.steps, "clocks": clk}
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    return line
+
+
+# ----------------------------------------------------------------------------------------------
 # more than 8 rows (one kernel pass per 8-row block)
 
 WIDE_ROWS = (16, 32, 64, 128)
@@ -925,7 +1263,8 @@ def main():
             print(json.dumps(line), flush=True)
         return
     world, rank, local = dist_setup(args.gpus)
-    run = {"sweep": run_ours, "attn_pairs": run_pairs, "wide_rows": run_wide}[args.workload]
+    run = {"sweep": run_ours, "attn_pairs": run_pairs, "wide_rows": run_wide,
+           "prologue_layers": run_prologue}[args.workload]
     line = run(args, world, rank, local)
     if line is not None and rank == 0:
         print(json.dumps(line), flush=True)

@@ -67,7 +67,8 @@ typedef enum {
     NVFP4_ERR_ALIGN = -4,     /* pointer or stride alignment (see each call) */
     NVFP4_ERR_ARCH = -5,      /* current device is not compute capability 10.0 (B200) */
     NVFP4_ERR_LAUNCH = -6,    /* the CUDA launch failed (cudaGetLastError) */
-    NVFP4_ERR_WORKSPACE = -7  /* workspace NULL, misaligned or smaller than required */
+    NVFP4_ERR_WORKSPACE = -7, /* workspace NULL, misaligned or smaller than required */
+    NVFP4_ERR_ALIAS = -8      /* a prologue's residual output overlaps what the call reads or y */
 } nvfp4_status;
 
 #define NVFP4_MAX_ROWS 128 /* rows of x (and y) per call */
@@ -179,6 +180,70 @@ int nvfp4_gemv_multi(const nvfp4_output_t* outputs, int count, const void* x, in
                      int m, int64_t k, void* workspace, size_t workspace_bytes, uint32_t flags,
                      cudaStream_t stream);
 
+/* Input prologues: the transform of x that the decode step runs just before a projection,
+ * applied while the GEMV stages x instead of in a launch of its own.  The decode plan launches
+ * them as residual_add_rms_norm / rms_norm (before the attention and FFN projections) and
+ * sigmoid_gate_mul (before the attention output projection) ("Blueprint - circuit executor"
+ * page for qwen3.8-27b-nvfp4 on GB10, table "Kernels the plan launches"; the page names them,
+ * the formulas are the standard RMS normalisation with a gain and the sigmoid output gate of
+ * gated attention).  The GEMV then runs on x', every weight of the call on the same x':
+ *
+ *   NVFP4_PROLOGUE_ADD_RMSNORM:   h[m][k]  = bf16_rn(x[m][k] + residual[m][k])
+ *                                 x'[m][k] = bf16_rn(h[m][k] * inv(m) * gamma[k]),
+ *                                 inv(m)   = 1 / sqrt(sum_k h[m][k]^2 / K + eps)
+ *                                 and h is written to residual_out when that is not NULL.
+ *   NVFP4_PROLOGUE_SIGMOID_GATE:  x'[m][k] = bf16_rn(x[m][k] / (1 + e^-gate[m][k]))
+ *
+ * in fp32 (h exactly rounded; the sum of squares in a fixed order).  gamma multiplies as given:
+ * a checkpoint that stores (gamma - 1) passes 1 + its weights.  Row invariance over M = 1..128
+ * and determinism hold as without a prologue, and h is bitwise the rounded sum.
+ */
+typedef enum {
+    NVFP4_PROLOGUE_NONE = 0,
+    NVFP4_PROLOGUE_ADD_RMSNORM = 1,
+    NVFP4_PROLOGUE_SIGMOID_GATE = 2
+} nvfp4_prologue_kind;
+
+typedef struct {
+    int32_t kind;            /* nvfp4_prologue_kind */
+    float eps;               /* ADD_RMSNORM: finite, >= 0 */
+    const void* residual;    /* ADD_RMSNORM: bf16 [M][ld_residual] */
+    int64_t ld_residual;
+    const void* gamma;       /* ADD_RMSNORM: bf16 [K] */
+    void* residual_out;      /* ADD_RMSNORM: bf16 [M][ld_residual_out] receives h, or NULL */
+    int64_t ld_residual_out;
+    const void* gate;        /* SIGMOID_GATE: bf16 [M][ld_gate] */
+    int64_t ld_gate;
+} nvfp4_prologue_t;
+
+/* nvfp4_gemv_ex, nvfp4_gemv_dual_ex and nvfp4_gemv_multi with an input prologue.  `prologue`
+ * is host memory read during the call only; NULL or kind NVFP4_PROLOGUE_NONE gives bitwise the
+ * call without one.  The prologue runs as a grid of its own ahead of the GEMV on `stream` (one
+ * CTA per row writes x' into the workspace, which must then hold nvfp4_workspace_bytes_wide(N,
+ * K, M) bytes; with NVFP4_FLAG_PREFETCH_WEIGHTS the GEMV's weights stream in meanwhile), so
+ * x' of a row is computed once and the GEMV's result is that of nvfp4_gemv on x'.  The
+ * prologue's arrays are device memory: every row 16-byte aligned (base 16-byte aligned,
+ * leading dimension >= K and a multiple of 8), like x.  residual_out may not
+ * overlap x, residual, gamma, the gate or any y (rows a launch reads while others write), and
+ * residual may not overlap y: NVFP4_ERR_ALIAS.  With NVFP4_FLAG_WIDE_TENSOR the tier's x pass
+ * applies the same prologue, and its rows are invariant over 9..128 as without one.
+ * Errors: those of the call without a prologue, and NVFP4_ERR_SHAPE (unknown kind, eps
+ * negative or not finite, a leading dimension < K), NVFP4_ERR_NULL (a required array NULL when
+ * K > 0), NVFP4_ERR_ALIGN, NVFP4_ERR_ALIAS, all checked before anything is enqueued. */
+int nvfp4_gemv_pro(const nvfp4_prologue_t* prologue, const uint8_t* w, const uint8_t* s,
+                   float global_scale, const void* x, int64_t ldx, void* y, int64_t ldy, int m,
+                   int64_t n, int64_t k, void* workspace, size_t workspace_bytes, uint32_t flags,
+                   cudaStream_t stream);
+int nvfp4_gemv_dual_pro(const nvfp4_prologue_t* prologue, const uint8_t* w_gate,
+                        const uint8_t* s_gate, float global_gate, const uint8_t* w_up,
+                        const uint8_t* s_up, float global_up, const void* x, int64_t ldx,
+                        void* y, int64_t ldy, int m, int64_t n, int64_t k, void* workspace,
+                        size_t workspace_bytes, uint32_t flags, cudaStream_t stream);
+int nvfp4_gemv_multi_pro(const nvfp4_prologue_t* prologue, const nvfp4_output_t* outputs,
+                         int count, const void* x, int64_t ldx, int m, int64_t k,
+                         void* workspace, size_t workspace_bytes, uint32_t flags,
+                         cudaStream_t stream);
+
 /* nvfp4_gemv for a caller that cannot provide a workspace.  The NVFP4 pages describe no such
  * call: it is a library convenience.  It serves callers that may not allocate device memory
  * and hold no buffer to lend: a plugin inside a host program that owns every device
@@ -208,11 +273,11 @@ int nvfp4_gemv_noalloc(const uint8_t* w, const uint8_t* s, float global_scale, c
                        int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
                        cudaStream_t stream);
 
-/* Workspace bytes of an nvfp4_gemv_ex or nvfp4_gemv_dual_ex call of M rows with
- * NVFP4_FLAG_WIDE_TENSOR: the nvfp4_workspace_bytes layout followed by the tier's scratch (fp32
- * partial sums of its split of K, an f16 copy of x with the rows' scales, and the dual's two
- * fp32 results; the size depends on N, K, M and the SM count).  Zero-filled before first use,
- * like any workspace.
+/* Workspace bytes of an nvfp4_gemv_ex / _pro or nvfp4_gemv_dual_ex / _pro call of M rows with
+ * NVFP4_FLAG_WIDE_TENSOR or an input prologue: the nvfp4_workspace_bytes layout followed by the
+ * larger of the tier's scratch (fp32 partial sums of its split of K, an f16 copy of x with the
+ * rows' scales, and the dual's two fp32 results; the size depends on N, K, M and the SM count)
+ * and the prologue's x' (M x K bf16).  Zero-filled before first use, like any workspace.
  * NVFP4_ERR_NULL, NVFP4_ERR_SHAPE (as nvfp4_gemv), NVFP4_ERR_ROWS, NVFP4_ERR_ARCH. */
 int nvfp4_workspace_bytes_wide(int64_t n, int64_t k, int m, size_t* bytes);
 

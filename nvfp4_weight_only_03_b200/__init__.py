@@ -8,6 +8,7 @@ missing or the device is not a B200 the calls raise.
     y = gemv(w, s, g, x)                      # y[m][n] = bf16(g * sum_k e2m1(w) e4m3(s) x)
     o = gemv_dual(wg, sg, gg, wu, su, gu, x)  # o = bf16(silu(gate) * up)
     k_, v_ = gemv_multi([(wk, sk, gk), (wv, sv, gv)], x)  # several outputs sharing x, one pass
+    q = gemv(w, s, g, x, prologue=AddRmsNorm(r, gamma, 1e-6, h))  # x' = rmsnorm(x + r) first
 
 w: uint8 [N][K/2] packed e2m1 (low nibble = even k), s: uint8 [N][K/16] e4m3 scale codes,
 g: float global scale, x: bfloat16 [M][K] (M = 1..128, one kernel pass per 8 rows; row stride
@@ -27,7 +28,7 @@ _lib = None
 
 STATUS = {0: "NVFP4_OK", -1: "NVFP4_ERR_NULL", -2: "NVFP4_ERR_SHAPE", -3: "NVFP4_ERR_ROWS",
           -4: "NVFP4_ERR_ALIGN", -5: "NVFP4_ERR_ARCH", -6: "NVFP4_ERR_LAUNCH",
-          -7: "NVFP4_ERR_WORKSPACE"}
+          -7: "NVFP4_ERR_WORKSPACE", -8: "NVFP4_ERR_ALIAS"}
 MAX_ROWS = 128
 PASS_ROWS = 8
 MAX_OUTPUTS = 4
@@ -46,6 +47,60 @@ class Output(ctypes.Structure):
     """nvfp4_output_t: one output of nvfp4_gemv_multi."""
     _fields_ = [("w", ctypes.c_void_p), ("s", ctypes.c_void_p), ("global_scale", ctypes.c_float),
                 ("y", ctypes.c_void_p), ("ldy", ctypes.c_int64), ("n", ctypes.c_int64)]
+
+
+class Prologue(ctypes.Structure):
+    """nvfp4_prologue_t: the transform of x a call applies before its GEMV."""
+    _fields_ = [("kind", ctypes.c_int32), ("eps", ctypes.c_float),
+                ("residual", ctypes.c_void_p), ("ld_residual", ctypes.c_int64),
+                ("gamma", ctypes.c_void_p),
+                ("residual_out", ctypes.c_void_p), ("ld_residual_out", ctypes.c_int64),
+                ("gate", ctypes.c_void_p), ("ld_gate", ctypes.c_int64)]
+
+
+PROLOGUE_NONE, PROLOGUE_ADD_RMSNORM, PROLOGUE_SIGMOID_GATE = 0, 1, 2
+
+
+def _rows_arg(t: torch.Tensor, m: int, k: int, name: str):
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16")
+    if t.dim() == 1:
+        t = t.unsqueeze(0)
+    if t.dim() != 2 or t.shape != (m, k) or t.stride(1) != 1:
+        raise ValueError(f"{name} must be [{m}][{k}] with unit inner stride")
+    return t, t.stride(0) if m > 1 else k
+
+
+class AddRmsNorm:
+    """Prologue: h = bf16(x + residual), x' = bf16(h / sqrt(mean(h^2) + eps) * gamma); h is
+    written to residual_out when given (it may not overlap x, residual, gamma or y)."""
+
+    def __init__(self, residual: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
+                 residual_out: torch.Tensor = None):
+        self.residual, self.gamma, self.eps, self.residual_out = residual, gamma, eps, residual_out
+
+    def struct(self, m: int, k: int) -> Prologue:
+        r, ldr = _rows_arg(self.residual, m, k, "residual")
+        if self.gamma.dtype != torch.bfloat16 or self.gamma.shape != (k,) or \
+                not self.gamma.is_contiguous():
+            raise ValueError(f"gamma must be contiguous bfloat16 [{k}]")
+        p = Prologue(kind=PROLOGUE_ADD_RMSNORM, eps=float(self.eps), residual=r.data_ptr(),
+                     ld_residual=ldr, gamma=self.gamma.data_ptr())
+        if self.residual_out is not None:
+            h, ldh = _rows_arg(self.residual_out, m, k, "residual_out")
+            p.residual_out, p.ld_residual_out = h.data_ptr(), ldh
+        return p
+
+
+class SigmoidGate:
+    """Prologue: x' = bf16(x * sigmoid(gate))."""
+
+    def __init__(self, gate: torch.Tensor):
+        self.gate = gate
+
+    def struct(self, m: int, k: int) -> Prologue:
+        t, ldt = _rows_arg(self.gate, m, k, "gate")
+        return Prologue(kind=PROLOGUE_SIGMOID_GATE, gate=t.data_ptr(), ld_gate=ldt)
 
 
 class PackInfo(ctypes.Structure):
@@ -83,13 +138,18 @@ def lib():
                                          i64, vp]
         L.nvfp4_gemv_multi.argtypes = [ctypes.POINTER(Output), c_int, vp, i64, c_int, i64, vp,
                                        sz, ctypes.c_uint32, vp]
+        pp = ctypes.POINTER(Prologue)
+        L.nvfp4_gemv_pro.argtypes = [pp] + L.nvfp4_gemv_ex.argtypes
+        L.nvfp4_gemv_dual_pro.argtypes = [pp] + L.nvfp4_gemv_dual_ex.argtypes
+        L.nvfp4_gemv_multi_pro.argtypes = [pp] + L.nvfp4_gemv_multi.argtypes
         L.nvfp4_workspace_error.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
         L.nvfp4_workspace_bytes_wide.argtypes = [i64, i64, c_int, ctypes.POINTER(sz)]
         L.nvfp4_status_string.argtypes = [c_int]
         L.nvfp4_status_string.restype = ctypes.c_char_p
         for f in (L.nvfp4_pack_info, L.nvfp4_workspace_bytes, L.nvfp4_gemv, L.nvfp4_gemv_dual,
                   L.nvfp4_gemv_ex, L.nvfp4_gemv_dual_ex, L.nvfp4_gemv_noalloc,
-                  L.nvfp4_gemv_multi, L.nvfp4_workspace_error, L.nvfp4_workspace_bytes_wide):
+                  L.nvfp4_gemv_multi, L.nvfp4_workspace_error, L.nvfp4_workspace_bytes_wide,
+                  L.nvfp4_gemv_pro, L.nvfp4_gemv_dual_pro, L.nvfp4_gemv_multi_pro):
             f.restype = c_int
         _lib = L
     return _lib
@@ -196,23 +256,29 @@ def wide_workspace(n: int, k: int, m: int, device=None) -> torch.Tensor:
 
 def gemv(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor, y: torch.Tensor = None,
          ws: torch.Tensor = None, stream=None, prefetch_weights: bool = False,
-         wide_tensor: bool = False) -> torch.Tensor:
+         wide_tensor: bool = False, prologue=None) -> torch.Tensor:
     """y[m][n] = bf16(g * sum_k e2m1(w[n][k]) * e4m3(s[n][k/16]) * x[m][k]) on the GPU.
 
     prefetch_weights: stream w and s before earlier work on the stream has finished
     (programmatic dependent launch); only valid when that work does not write w or s.
     wide_tensor: calls of 9..128 rows run on the tensor-core tier (one pass over the weights;
-    rows invariant over 9..128, equal to 1..8-row calls within the tolerance)."""
+    rows invariant over 9..128, equal to 1..8-row calls within the tolerance).
+    prologue: AddRmsNorm or SigmoidGate, applied to x inside the call (its x' lives in the
+    workspace, so a caller's ws must hold workspace_bytes_wide(n, k, m))."""
     n, k = _weight_args(w, s)
     x, m, ldx = _x_args(x, k)
+    pro = None if prologue is None else prologue.struct(m, k)
     y, ldy = _out(y, m, n, x)
     if ws is None:
-        ws = wide_workspace(n, k, m, x.device) if wide_tensor else workspace(x.device)
+        ws = wide_workspace(n, k, m, x.device) if (wide_tensor or pro) else workspace(x.device)
     flags = (FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0) | \
         (FLAG_WIDE_TENSOR if wide_tensor else 0)
-    st = lib().nvfp4_gemv_ex(w.data_ptr(), s.data_ptr(), float(g), x.data_ptr(), ldx,
-                             y.data_ptr(), ldy, m, n, k, ws.data_ptr(), ws.numel(), flags,
-                             _stream(stream))
+    args = (w.data_ptr(), s.data_ptr(), float(g), x.data_ptr(), ldx, y.data_ptr(), ldy, m, n, k,
+            ws.data_ptr(), ws.numel(), flags, _stream(stream))
+    if pro is None:
+        st = lib().nvfp4_gemv_ex(*args)
+    else:
+        st = lib().nvfp4_gemv_pro(ctypes.byref(pro), *args)
     _check(st, "nvfp4_gemv")
     return y
 
@@ -234,32 +300,38 @@ def gemv_noalloc(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor,
 def gemv_dual(wg: torch.Tensor, sg: torch.Tensor, gg: float, wu: torch.Tensor, su: torch.Tensor,
               gu: float, x: torch.Tensor, y: torch.Tensor = None, ws: torch.Tensor = None,
               stream=None, prefetch_weights: bool = False,
-              wide_tensor: bool = False) -> torch.Tensor:
+              wide_tensor: bool = False, prologue=None) -> torch.Tensor:
     """o[m][n] = bf16(silu(gate) * up), gate/up the two NVFP4 GEMVs of the same x.
 
     wide_tensor: calls of 9..128 rows run gate and up on the tensor-core tier, kept in fp32
-    and combined by one final pass."""
+    and combined by one final pass.  prologue: as for gemv."""
     n, k = _weight_args(wg, sg)
     if _weight_args(wu, su) != (n, k):
         raise ValueError("gate and up weights must have the same shape")
     x, m, ldx = _x_args(x, k)
+    pro = None if prologue is None else prologue.struct(m, k)
     y, ldy = _out(y, m, n, x)
     if ws is None:
-        ws = wide_workspace(n, k, m, x.device) if wide_tensor else workspace(x.device)
+        ws = wide_workspace(n, k, m, x.device) if (wide_tensor or pro) else workspace(x.device)
     flags = (FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0) | \
         (FLAG_WIDE_TENSOR if wide_tensor else 0)
-    st = lib().nvfp4_gemv_dual_ex(wg.data_ptr(), sg.data_ptr(), float(gg), wu.data_ptr(),
-                                  su.data_ptr(), float(gu), x.data_ptr(), ldx, y.data_ptr(), ldy,
-                                  m, n, k, ws.data_ptr(), ws.numel(), flags, _stream(stream))
+    args = (wg.data_ptr(), sg.data_ptr(), float(gg), wu.data_ptr(), su.data_ptr(), float(gu),
+            x.data_ptr(), ldx, y.data_ptr(), ldy, m, n, k, ws.data_ptr(), ws.numel(), flags,
+            _stream(stream))
+    if pro is None:
+        st = lib().nvfp4_gemv_dual_ex(*args)
+    else:
+        st = lib().nvfp4_gemv_dual_pro(ctypes.byref(pro), *args)
     _check(st, "nvfp4_gemv_dual")
     return y
 
 
 def gemv_multi(weights, x: torch.Tensor, ys=None, ws: torch.Tensor = None, stream=None,
-               prefetch_weights: bool = False) -> list:
+               prefetch_weights: bool = False, prologue=None) -> list:
     """Several GEMVs sharing x in one pass (nvfp4_gemv_multi): weights is a list of up to
     MAX_OUTPUTS (w, s, g) triples with the same K; returns [y_0, y_1, ...], y_o the GEMV of
-    weight o as gemv computes it.  ys: optional preallocated outputs, one per weight."""
+    weight o as gemv computes it.  ys: optional preallocated outputs, one per weight.
+    prologue: as for gemv, applied once to the shared x."""
     weights = list(weights)
     if not 1 <= len(weights) <= MAX_OUTPUTS:
         raise ValueError(f"1..{MAX_OUTPUTS} weights, got {len(weights)}")
@@ -268,6 +340,7 @@ def gemv_multi(weights, x: torch.Tensor, ys=None, ws: torch.Tensor = None, strea
     if any(kk != k for _, kk in shapes):
         raise ValueError("all weights must have the same K")
     x, m, ldx = _x_args(x, k)
+    pro = None if prologue is None else prologue.struct(m, k)
     ys = [None] * len(weights) if ys is None else list(ys)
     if len(ys) != len(weights):
         raise ValueError("one output per weight")
@@ -278,9 +351,15 @@ def gemv_multi(weights, x: torch.Tensor, ys=None, ws: torch.Tensor = None, strea
         result.append(y)
         outs[o].w, outs[o].s, outs[o].global_scale = w.data_ptr(), s.data_ptr(), float(g)
         outs[o].y, outs[o].ldy, outs[o].n = y.data_ptr(), ldy, n
-    ws = workspace(x.device) if ws is None else ws
+    if ws is None:
+        ws = wide_workspace(max(n for n, _ in shapes), k, m, x.device) if pro else \
+            workspace(x.device)
     flags = FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0
-    st = lib().nvfp4_gemv_multi(outs, len(weights), x.data_ptr(), ldx, m, k, ws.data_ptr(),
-                                ws.numel(), flags, _stream(stream))
+    args = (outs, len(weights), x.data_ptr(), ldx, m, k, ws.data_ptr(), ws.numel(), flags,
+            _stream(stream))
+    if pro is None:
+        st = lib().nvfp4_gemv_multi(*args)
+    else:
+        st = lib().nvfp4_gemv_multi_pro(ctypes.byref(pro), *args)
     _check(st, "nvfp4_gemv_multi")
     return result

@@ -7,7 +7,8 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRCS = [os.path.join(HERE, "csrc", "nvfp4_gemv.cu"), os.path.join(HERE, "csrc", "nvfp4_gemv_tc.cu")]
-HDRS = [os.path.join(ROOT, "include", "nvfp4.h"), os.path.join(HERE, "csrc", "nvfp4_tc.h")]
+HDRS = [os.path.join(ROOT, "include", "nvfp4.h"), os.path.join(HERE, "csrc", "nvfp4_tc.h"),
+        os.path.join(HERE, "csrc", "nvfp4_prologue.h")]
 LIB = os.path.join(HERE, "libnvfp4gemv.so")
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -53,6 +53,7 @@
 #include <string.h>
 
 #include "nvfp4.h"
+#include "nvfp4_prologue.h"
 #include "nvfp4_tc.h"
 
 namespace {
@@ -731,6 +732,98 @@ struct DeviceInfo {
     int sms = 0;
 };
 DeviceInfo g_dev[64];
+// ------------------------------------------------------------------------------------------
+// The input prologue as a pass of its own, ahead of the GEMV on the same stream: one CTA per row
+// of x writes x' (and h).  A row-wide reduction (the RMS norm) cannot be split over the GEMV's
+// CTAs without each of them reading the whole row (148 copies of it through L2 per launch) or a
+// grid-wide barrier; one small grid chained by programmatic dependent launch costs less.  The
+// arithmetic is that of nvfp4_prologue.h; thread t of a row takes 16-byte chunks t, t + 512, ...
+// in order, then a fixed xor tree per warp and the warps in order.
+
+constexpr int kProThreads = 512;
+constexpr int kProKeep = 4;  // chunks a thread keeps in registers between the two passes
+
+__global__ void __launch_bounds__(kProThreads)
+    nvfp4_prologue_kernel(const nvfp4_pro::Prologue pro, const uint16_t* __restrict__ x,
+                          int64_t ldx, int64_t k, uint16_t* __restrict__ xo) {
+    pdl_launch_dependents();
+    pdl_wait();  // x and the prologue's arrays may come from the preceding kernel
+    __shared__ float s_red[kProThreads / 32];
+    __shared__ float s_inv;
+    const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t nch = k >> 3;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + m * ldx);
+    const uint4* ar = reinterpret_cast<const uint4*>(pro.in + m * pro.ld_in);
+    uint4* outr = reinterpret_cast<uint4*>(xo + m * k);
+    constexpr int64_t kRound = (int64_t)kProKeep * kProThreads;
+    if (pro.kind == NVFP4_PROLOGUE_SIGMOID_GATE) {
+        for (int64_t base = 0; base < nch; base += kRound) {
+            uint4 xv[kProKeep], tv[kProKeep];
+#pragma unroll
+            for (int u = 0; u < kProKeep; ++u) {
+                const int64_t j = base + tid + u * kProThreads;
+                if (j < nch) {
+                    xv[u] = xr[j];
+                    tv[u] = ar[j];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kProKeep; ++u) {
+                const int64_t j = base + tid + u * kProThreads;
+                if (j < nch) outr[j] = nvfp4_pro::gate_8(xv[u], tv[u]);
+            }
+        }
+        return;
+    }
+    const uint4* gr = reinterpret_cast<const uint4*>(pro.gamma);
+    uint4* hr = pro.hout ? reinterpret_cast<uint4*>(pro.hout + m * pro.ldh) : nullptr;
+    const bool keep = nch <= kRound;  // one round: h and gamma stay in registers
+    uint4 hv[kProKeep], gv[kProKeep];
+    float ss = 0.f;
+    for (int64_t base = 0; base < nch; base += kRound) {
+        uint4 xv[kProKeep], rv[kProKeep];
+#pragma unroll
+        for (int u = 0; u < kProKeep; ++u) {
+            const int64_t j = base + tid + u * kProThreads;
+            if (j < nch) {
+                xv[u] = xr[j];
+                rv[u] = ar[j];
+                if (keep) gv[u] = gr[j];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kProKeep; ++u) {
+            const int64_t j = base + tid + u * kProThreads;
+            if (j < nch) {
+                hv[u] = nvfp4_pro::add_8(xv[u], rv[u]);
+                ss = nvfp4_pro::sum_squares_8(hv[u], ss);
+                if (hr) hr[j] = hv[u];
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+    if (lane == 0) s_red[warp] = ss;
+    __syncthreads();
+    if (tid == 0) {
+        float t = 0.f;
+        for (int w = 0; w < kProThreads / 32; ++w) t += s_red[w];
+        s_inv = nvfp4_pro::rms_inverse(t, k, pro.eps);
+    }
+    __syncthreads();
+    const float inv = s_inv;
+    if (keep) {
+#pragma unroll
+        for (int u = 0; u < kProKeep; ++u) {
+            const int64_t j = tid + u * kProThreads;
+            if (j < nch) outr[j] = nvfp4_pro::scale_8(hv[u], gv[u], inv);
+        }
+    } else {
+        for (int64_t j = tid; j < nch; j += kProThreads)
+            outr[j] = nvfp4_pro::norm_8(xr[j], ar[j], gr[j], inv);
+    }
+}
+
 bool g_attr_set[3][64];  // single, dual, multi
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -811,6 +904,60 @@ int check_weight(const uint8_t* w, const uint8_t* s) {
     if (misaligned(w, 16) || misaligned(s, 2)) return NVFP4_ERR_ALIGN;
     return NVFP4_OK;
 }
+
+// Bytes [lo, hi) spanned by m rows of `cols` bf16 values at row stride ld (m, cols > 0).
+struct Range {
+    uintptr_t lo, hi;
+};
+
+Range rows_range(const void* p, int m, int64_t ld, int64_t cols) {
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+    return {lo, lo + (uintptr_t)(((int64_t)(m - 1) * ld + cols) * 2)};
+}
+
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+// A caller's prologue checked against the call's x (M x K) and its outputs `ys`, turned into
+// the kernels' form (kind NONE for NULL).
+int check_pro(const nvfp4_prologue_t* pp, const void* x, int64_t ldx, int m, int64_t k,
+              const Range* ys, int ny, nvfp4_pro::Prologue* out) {
+    memset(out, 0, sizeof(*out));
+    if (!pp || pp->kind == NVFP4_PROLOGUE_NONE) return NVFP4_OK;
+    const bool norm = pp->kind == NVFP4_PROLOGUE_ADD_RMSNORM;
+    if (!norm && pp->kind != NVFP4_PROLOGUE_SIGMOID_GATE) return NVFP4_ERR_SHAPE;
+    if (norm && !(pp->eps >= 0.0f && pp->eps <= 3.402823466e38f)) return NVFP4_ERR_SHAPE;
+    out->kind = pp->kind;
+    out->eps = norm ? pp->eps : 0.0f;
+    if (m <= 0 || k <= 0) return NVFP4_OK;  // nothing to read or write
+    const void* in = norm ? pp->residual : pp->gate;
+    const int64_t ld_in = norm ? pp->ld_residual : pp->ld_gate;
+    void* hout = norm ? pp->residual_out : nullptr;
+    if (!in || (norm && !pp->gamma)) return NVFP4_ERR_NULL;
+    if (ld_in < k || (hout && pp->ld_residual_out < k)) return NVFP4_ERR_SHAPE;
+    if ((ld_in % 8) != 0 || misaligned(in, 16) || (norm && misaligned(pp->gamma, 16)))
+        return NVFP4_ERR_ALIGN;
+    if (hout && ((pp->ld_residual_out % 8) != 0 || misaligned(hout, 16))) return NVFP4_ERR_ALIGN;
+    // residual_out is written while other CTAs read x, residual and gamma; y is written while
+    // they read the residual or the gate
+    const Range rin = rows_range(in, m, ld_in, k);
+    for (int i = 0; i < ny; ++i)
+        if (overlap(rin, ys[i])) return NVFP4_ERR_ALIAS;
+    if (hout) {
+        const Range ro = rows_range(hout, m, pp->ld_residual_out, k);
+        if (overlap(ro, rows_range(x, m, ldx, k)) || overlap(ro, rin) ||
+            overlap(ro, rows_range(pp->gamma, 1, k, k)))
+            return NVFP4_ERR_ALIAS;
+        for (int i = 0; i < ny; ++i)
+            if (overlap(ro, ys[i])) return NVFP4_ERR_ALIAS;
+    }
+    out->in = static_cast<const uint16_t*>(in);
+    out->ld_in = ld_in;
+    out->gamma = norm ? static_cast<const uint16_t*>(pp->gamma) : nullptr;
+    out->hout = static_cast<uint16_t*>(hout);
+    out->ldh = hout ? pp->ld_residual_out : 0;
+    return NVFP4_OK;
+}
+
 
 // 2-D map over a [rows][cols] byte matrix with row stride = cols: box = box_cols bytes x
 // box_rows rows, zero fill outside.
@@ -1024,6 +1171,46 @@ int launch(const uint8_t* const* w, const uint8_t* const* s, const float* gs, co
     return NVFP4_OK;
 }
 
+// Bytes the prologue pass adds after the workspace layout: x' of m rows, row stride k.
+size_t prologue_scratch_bytes(int m, int64_t k) {
+    return ((size_t)m * (size_t)k * 2 + 255) / 256 * 256;
+}
+
+// Enqueues the prologue pass of a call, when it has one, and points x / ldx at its output
+// (x' in the workspace after its layout).  Nothing is enqueued when the workspace is short.
+int prologue_pass(const nvfp4_pro::Prologue& pro, const void** x, int64_t* ldx, int m, int64_t k,
+                  void* ws, size_t ws_bytes, uint32_t flags, cudaStream_t stream) {
+    if (pro.kind == NVFP4_PROLOGUE_NONE || m == 0 || k == 0) return NVFP4_OK;
+    int dev = 0;
+    DeviceInfo* di = nullptr;
+    int st = device_info(&dev, &di);
+    if (st != NVFP4_OK) return st;
+    size_t flags_off, partial_off;
+    const size_t base = workspace_layout(di->sms, &flags_off, &partial_off);
+    if (ws_bytes < base + prologue_scratch_bytes(m, k)) return NVFP4_ERR_WORKSPACE;
+    uint16_t* xo = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + base);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)m);
+    cfg.blockDim = dim3(kProThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    if (flags & NVFP4_FLAG_PREFETCH_WEIGHTS) {
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    if (cudaLaunchKernelEx(&cfg, nvfp4_prologue_kernel, pro, static_cast<const uint16_t*>(*x),
+                           *ldx, k, xo) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_LAUNCH;
+    }
+    *x = xo;
+    *ldx = k;
+    return NVFP4_OK;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------------------------------
@@ -1074,12 +1261,17 @@ int nvfp4_workspace_bytes(size_t* bytes) {
     return NVFP4_OK;
 }
 
-int nvfp4_gemv_ex(const uint8_t* w, const uint8_t* s, float global_scale, const void* x,
-                  int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
-                  void* workspace, size_t workspace_bytes, uint32_t flags, cudaStream_t stream) {
+int nvfp4_gemv_pro(const nvfp4_prologue_t* prologue, const uint8_t* w, const uint8_t* s,
+                   float global_scale, const void* x, int64_t ldx, void* y, int64_t ldy, int m,
+                   int64_t n, int64_t k, void* workspace, size_t workspace_bytes, uint32_t flags,
+                   cudaStream_t stream) {
     bool noop = false;
     int st = check_common(x, ldx, y, ldy, m, n, k, workspace, flags, &noop);
-    if (st != NVFP4_OK || noop) return st;
+    if (st != NVFP4_OK) return st;
+    nvfp4_pro::Prologue pro;
+    const Range yr = noop ? Range{0, 0} : rows_range(y, m, ldy, n);
+    if ((st = check_pro(prologue, x, ldx, m, k, &yr, noop ? 0 : 1, &pro)) != NVFP4_OK) return st;
+    if (noop) return NVFP4_OK;
     if (k > 0 && (st = check_weight(w, s)) != NVFP4_OK) return st;
     if ((flags & NVFP4_FLAG_WIDE_TENSOR) && m > NVFP4_PASS_ROWS && k > 0 &&
         nvfp4_tc::usable(s, k)) {
@@ -1089,8 +1281,11 @@ int nvfp4_gemv_ex(const uint8_t* w, const uint8_t* s, float global_scale, const 
         size_t flags_off, partial_off;
         const size_t base = workspace_layout(di->sms, &flags_off, &partial_off);
         return nvfp4_tc::launch(g_encode, di->sms, w, s, global_scale, x, ldx, y, ldy, m, n, k,
-                                workspace, workspace_bytes, base, stream);
+                                pro, workspace, workspace_bytes, base, stream);
     }
+    if ((st = prologue_pass(pro, &x, &ldx, m, k, workspace, workspace_bytes, flags, stream)) !=
+        NVFP4_OK)
+        return st;
     const uint8_t* ws_[1] = {w};
     const uint8_t* ss_[1] = {s};
     const float gs[1] = {global_scale};
@@ -1098,11 +1293,18 @@ int nvfp4_gemv_ex(const uint8_t* w, const uint8_t* s, float global_scale, const 
                          flags, stream);
 }
 
+int nvfp4_gemv_ex(const uint8_t* w, const uint8_t* s, float global_scale, const void* x,
+                  int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
+                  void* workspace, size_t workspace_bytes, uint32_t flags, cudaStream_t stream) {
+    return nvfp4_gemv_pro(nullptr, w, s, global_scale, x, ldx, y, ldy, m, n, k, workspace,
+                          workspace_bytes, flags, stream);
+}
+
 int nvfp4_gemv(const uint8_t* w, const uint8_t* s, float global_scale, const void* x,
                int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* workspace,
                size_t workspace_bytes, cudaStream_t stream) {
-    return nvfp4_gemv_ex(w, s, global_scale, x, ldx, y, ldy, m, n, k, workspace,
-                         workspace_bytes, 0u, stream);
+    return nvfp4_gemv_pro(nullptr, w, s, global_scale, x, ldx, y, ldy, m, n, k, workspace,
+                          workspace_bytes, 0u, stream);
 }
 
 int nvfp4_gemv_noalloc(const uint8_t* w, const uint8_t* s, float global_scale, const void* x,
@@ -1142,14 +1344,18 @@ int nvfp4_gemv_noalloc(const uint8_t* w, const uint8_t* s, float global_scale, c
                          stream);
 }
 
-int nvfp4_gemv_dual_ex(const uint8_t* w_gate, const uint8_t* s_gate, float global_gate,
-                       const uint8_t* w_up, const uint8_t* s_up, float global_up, const void* x,
-                       int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
-                       void* workspace, size_t workspace_bytes, uint32_t flags,
-                       cudaStream_t stream) {
+int nvfp4_gemv_dual_pro(const nvfp4_prologue_t* prologue, const uint8_t* w_gate,
+                        const uint8_t* s_gate, float global_gate, const uint8_t* w_up,
+                        const uint8_t* s_up, float global_up, const void* x, int64_t ldx,
+                        void* y, int64_t ldy, int m, int64_t n, int64_t k, void* workspace,
+                        size_t workspace_bytes, uint32_t flags, cudaStream_t stream) {
     bool noop = false;
     int st = check_common(x, ldx, y, ldy, m, n, k, workspace, flags, &noop);
-    if (st != NVFP4_OK || noop) return st;
+    if (st != NVFP4_OK) return st;
+    nvfp4_pro::Prologue pro;
+    const Range yr = noop ? Range{0, 0} : rows_range(y, m, ldy, n);
+    if ((st = check_pro(prologue, x, ldx, m, k, &yr, noop ? 0 : 1, &pro)) != NVFP4_OK) return st;
+    if (noop) return NVFP4_OK;
     if (k > 0) {
         if ((st = check_weight(w_gate, s_gate)) != NVFP4_OK) return st;
         if ((st = check_weight(w_up, s_up)) != NVFP4_OK) return st;
@@ -1162,9 +1368,12 @@ int nvfp4_gemv_dual_ex(const uint8_t* w_gate, const uint8_t* s_gate, float globa
         size_t flags_off, partial_off;
         const size_t base = workspace_layout(di->sms, &flags_off, &partial_off);
         return nvfp4_tc::launch_dual(g_encode, di->sms, w_gate, s_gate, global_gate, w_up, s_up,
-                                     global_up, x, ldx, y, ldy, m, n, k, workspace,
+                                     global_up, x, ldx, y, ldy, m, n, k, pro, workspace,
                                      workspace_bytes, base, stream);
     }
+    if ((st = prologue_pass(pro, &x, &ldx, m, k, workspace, workspace_bytes, flags, stream)) !=
+        NVFP4_OK)
+        return st;
     const uint8_t* ws_[2] = {w_gate, w_up};
     const uint8_t* ss_[2] = {s_gate, s_up};
     const float gs[2] = {global_gate, global_up};
@@ -1172,20 +1381,31 @@ int nvfp4_gemv_dual_ex(const uint8_t* w_gate, const uint8_t* s_gate, float globa
                         stream);
 }
 
+int nvfp4_gemv_dual_ex(const uint8_t* w_gate, const uint8_t* s_gate, float global_gate,
+                       const uint8_t* w_up, const uint8_t* s_up, float global_up, const void* x,
+                       int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
+                       void* workspace, size_t workspace_bytes, uint32_t flags,
+                       cudaStream_t stream) {
+    return nvfp4_gemv_dual_pro(nullptr, w_gate, s_gate, global_gate, w_up, s_up, global_up, x,
+                               ldx, y, ldy, m, n, k, workspace, workspace_bytes, flags, stream);
+}
+
 int nvfp4_gemv_dual(const uint8_t* w_gate, const uint8_t* s_gate, float global_gate,
                     const uint8_t* w_up, const uint8_t* s_up, float global_up, const void* x,
                     int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
                     void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-    return nvfp4_gemv_dual_ex(w_gate, s_gate, global_gate, w_up, s_up, global_up, x, ldx, y, ldy,
-                              m, n, k, workspace, workspace_bytes, 0u, stream);
+    return nvfp4_gemv_dual_pro(nullptr, w_gate, s_gate, global_gate, w_up, s_up, global_up, x,
+                               ldx, y, ldy, m, n, k, workspace, workspace_bytes, 0u, stream);
 }
 
-int nvfp4_gemv_multi(const nvfp4_output_t* outputs, int count, const void* x, int64_t ldx,
-                     int m, int64_t k, void* workspace, size_t workspace_bytes, uint32_t flags,
-                     cudaStream_t stream) {
+int nvfp4_gemv_multi_pro(const nvfp4_prologue_t* prologue, const nvfp4_output_t* outputs,
+                         int count, const void* x, int64_t ldx, int m, int64_t k,
+                         void* workspace, size_t workspace_bytes, uint32_t flags,
+                         cudaStream_t stream) {
     if (!outputs) return NVFP4_ERR_NULL;
     if (count < 1 || count > NVFP4_MAX_OUTPUTS) return NVFP4_ERR_SHAPE;
     Span sp[kMaxOutputs];
+    Range yr[kMaxOutputs];
     int used = 0;
     for (int o = 0; o < count; ++o) {
         const nvfp4_output_t& a = outputs[o];
@@ -1194,6 +1414,7 @@ int nvfp4_gemv_multi(const nvfp4_output_t* outputs, int count, const void* x, in
         if (st != NVFP4_OK) return st;
         if (noop) continue;  // M == 0 or no rows: nothing to write
         if (k > 0 && (st = check_weight(a.w, a.s)) != NVFP4_OK) return st;
+        yr[used] = rows_range(a.y, m, a.ldy, a.n);
         Span& b = sp[used++];
         memset(&b, 0, sizeof(b));
         b.w[0] = a.w;
@@ -1203,11 +1424,17 @@ int nvfp4_gemv_multi(const nvfp4_output_t* outputs, int count, const void* x, in
         b.ldy = a.ldy;
         b.n = a.n;
     }
+    nvfp4_pro::Prologue pro;
+    int st = check_pro(prologue, x, ldx, m, k, yr, used, &pro);
+    if (st != NVFP4_OK) return st;
     if (used == 0) return NVFP4_OK;
     int dev = 0;
     DeviceInfo* di = nullptr;
-    int st = device_info(&dev, &di);
+    st = device_info(&dev, &di);
     if (st != NVFP4_OK) return st;
+    if ((st = prologue_pass(pro, &x, &ldx, m, k, workspace, workspace_bytes, flags, stream)) !=
+        NVFP4_OK)
+        return st;
     using C = Cfg<false>;
     int64_t groups = 0;
     for (int o = 0; o < used; ++o) groups += (sp[o].n + C::kRows - 1) / C::kRows;
@@ -1230,6 +1457,13 @@ int nvfp4_gemv_multi(const nvfp4_output_t* outputs, int count, const void* x, in
     return NVFP4_OK;
 }
 
+int nvfp4_gemv_multi(const nvfp4_output_t* outputs, int count, const void* x, int64_t ldx,
+                     int m, int64_t k, void* workspace, size_t workspace_bytes, uint32_t flags,
+                     cudaStream_t stream) {
+    return nvfp4_gemv_multi_pro(nullptr, outputs, count, x, ldx, m, k, workspace,
+                                workspace_bytes, flags, stream);
+}
+
 int nvfp4_workspace_bytes_wide(int64_t n, int64_t k, int m, size_t* bytes) {
     if (!bytes) return NVFP4_ERR_NULL;
     if (n < 0 || k < 0 || (k % 32) != 0 || k > kMaxK) return NVFP4_ERR_SHAPE;
@@ -1239,8 +1473,9 @@ int nvfp4_workspace_bytes_wide(int64_t n, int64_t k, int m, size_t* bytes) {
     int st = device_info(&dev, &di);
     if (st != NVFP4_OK) return st;
     size_t flags_off, partial_off;
-    *bytes = workspace_layout(di->sms, &flags_off, &partial_off) +
-             (m > NVFP4_PASS_ROWS ? nvfp4_tc::scratch_bytes(n, k, m, di->sms) : 0);
+    const size_t tier = m > NVFP4_PASS_ROWS ? nvfp4_tc::scratch_bytes(n, k, m, di->sms) : 0;
+    const size_t pro = prologue_scratch_bytes(m, k);
+    *bytes = workspace_layout(di->sms, &flags_off, &partial_off) + (tier > pro ? tier : pro);
     return NVFP4_OK;
 }
 
@@ -1269,6 +1504,7 @@ const char* nvfp4_status_string(int status) {
         case NVFP4_ERR_ARCH: return "NVFP4_ERR_ARCH";
         case NVFP4_ERR_LAUNCH: return "NVFP4_ERR_LAUNCH";
         case NVFP4_ERR_WORKSPACE: return "NVFP4_ERR_WORKSPACE";
+        case NVFP4_ERR_ALIAS: return "NVFP4_ERR_ALIAS";
         default: return "NVFP4_ERR_UNKNOWN";
     }
 }

@@ -407,22 +407,49 @@ __global__ void nvfp4_tc_silu_mul(const float* __restrict__ gate, const float* _
     y[(int64_t)mm * ldy + nn] = f2bf(a / (1.0f + expf(-a)) * b);
 }
 
-// The f16 copy of x: row m scaled by 2^e(m) so that its largest magnitude lands in
-// [2^14, 2^15) (exact for every bf16 value at most 2^24 times smaller), and 2^-e(m).
-// One block per row, 16-byte accesses (K % 256 == 0, 16-byte aligned rows).
+// The f16 copy of x (after the call's prologue, if any): row m scaled by 2^e(m) so that its
+// largest magnitude lands in [2^14, 2^15) (exact for every bf16 value at most 2^24 times
+// smaller), and 2^-e(m).  One block per row, 16-byte accesses (K % 256 == 0, 16-byte aligned
+// rows).  With the residual-add + RMS-norm prologue the block first sums h^2 over the row (a
+// fixed xor tree per warp, then the warps in order) and writes h.
 __global__ void __launch_bounds__(512) nvfp4_tc_prep(const uint16_t* __restrict__ x, int64_t ldx,
-                                                     int64_t k, uint16_t* x16, float* descale) {
+                                                     int64_t k, uint16_t* x16, float* descale,
+                                                     const nvfp4_pro::Prologue pro) {
     const int m = blockIdx.x;
     const uint4* row = reinterpret_cast<const uint4*>(x + (int64_t)m * ldx);
     const int64_t k8 = k / 8;
+    __shared__ uint32_t red[32];
+    __shared__ float fred[32];
+    float inv = 0.f;
+    if (pro.kind == NVFP4_PROLOGUE_ADD_RMSNORM) {
+        const uint4* rr = reinterpret_cast<const uint4*>(pro.in + (int64_t)m * pro.ld_in);
+        uint4* hr = pro.hout ? reinterpret_cast<uint4*>(pro.hout + (int64_t)m * pro.ldh) : nullptr;
+        float ss = 0.f;
+        for (int64_t i = threadIdx.x; i < k8; i += blockDim.x) {
+            const uint4 h = nvfp4_pro::add_8(row[i], rr[i]);
+            ss = nvfp4_pro::sum_squares_8(h, ss);
+            if (hr) hr[i] = h;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+        if ((threadIdx.x & 31) == 0) fred[threadIdx.x >> 5] = ss;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float t = 0.f;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += fred[w];
+            fred[0] = nvfp4_pro::rms_inverse(t, k, pro.eps);
+        }
+        __syncthreads();
+        inv = fred[0];
+    }
     uint32_t a = 0;
     for (int64_t i = threadIdx.x; i < k8; i += blockDim.x) {
-        const uint4 v = row[i];
+        uint4 v = row[i];
+        if (pro.kind != NVFP4_PROLOGUE_NONE) v = nvfp4_pro::apply_8(pro, v, m, 8 * i, inv);
         a = max(a, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
                             __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
     }
     a = max(a & 0xFFFFu, a >> 16);
-    __shared__ uint32_t red[32];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
@@ -442,7 +469,8 @@ __global__ void __launch_bounds__(512) nvfp4_tc_prep(const uint16_t* __restrict_
     if (threadIdx.x == 0) descale[m] = __uint_as_float((uint32_t)(127 - e) << 23);
     uint4* out = reinterpret_cast<uint4*>(x16 + (int64_t)m * k);
     for (int64_t i = threadIdx.x; i < k8; i += blockDim.x) {
-        const uint4 v = row[i];
+        uint4 v = row[i];
+        if (pro.kind != NVFP4_PROLOGUE_NONE) v = nvfp4_pro::apply_8(pro, v, m, 8 * i, inv);
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
         uint32_t h4[4];
 #pragma unroll
@@ -608,8 +636,9 @@ static int enqueue_weight(EncodeFn encode, int sms, const uint8_t* w, const uint
 }
 
 int launch(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g, const void* x,
-           int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws,
-           size_t ws_bytes, size_t scratch_off, cudaStream_t stream) {
+           int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
+           const nvfp4_pro::Prologue& pro, void* ws, size_t ws_bytes, size_t scratch_off,
+           cudaStream_t stream) {
     if (ws_bytes < scratch_off + scratch_bytes(n, k, m, sms)) return NVFP4_ERR_WORKSPACE;
     int st = set_attr();
     if (st != NVFP4_OK) return st;
@@ -617,7 +646,8 @@ int launch(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g
     char* const base = static_cast<char*>(ws) + scratch_off;
     uint16_t* const x16 = reinterpret_cast<uint16_t*>(base + sc.x16);
     float* const descale = reinterpret_cast<float*>(base + sc.descale);
-    nvfp4_tc_prep<<<m, 512, 0, stream>>>(static_cast<const uint16_t*>(x), ldx, k, x16, descale);
+    nvfp4_tc_prep<<<m, 512, 0, stream>>>(static_cast<const uint16_t*>(x), ldx, k, x16, descale,
+                                         pro);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
     return enqueue_weight(encode, sms, w, s, g, x16, descale,
                           reinterpret_cast<float*>(base + sc.partial), m, n, k,
@@ -626,8 +656,8 @@ int launch(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g
 
 int launch_dual(EncodeFn encode, int sms, const uint8_t* wg, const uint8_t* sg, float gg,
                 const uint8_t* wu, const uint8_t* su, float gu, const void* x, int64_t ldx,
-                void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws, size_t ws_bytes,
-                size_t scratch_off, cudaStream_t stream) {
+                void* y, int64_t ldy, int m, int64_t n, int64_t k, const nvfp4_pro::Prologue& pro,
+                void* ws, size_t ws_bytes, size_t scratch_off, cudaStream_t stream) {
     if (ws_bytes < scratch_off + scratch_bytes(n, k, m, sms)) return NVFP4_ERR_WORKSPACE;
     int st = set_attr();
     if (st != NVFP4_OK) return st;
@@ -639,7 +669,8 @@ int launch_dual(EncodeFn encode, int sms, const uint8_t* wg, const uint8_t* sg, 
     float* const gate = reinterpret_cast<float*>(base + sc.gate);
     float* const up = reinterpret_cast<float*>(base + sc.up);
     int32_t* const error = static_cast<int32_t*>(ws);
-    nvfp4_tc_prep<<<m, 512, 0, stream>>>(static_cast<const uint16_t*>(x), ldx, k, x16, descale);
+    nvfp4_tc_prep<<<m, 512, 0, stream>>>(static_cast<const uint16_t*>(x), ldx, k, x16, descale,
+                                         pro);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
     if ((st = enqueue_weight(encode, sms, wg, sg, gg, x16, descale, partial, m, n, k, nullptr, 0,
                              gate, error, stream)) != NVFP4_OK)

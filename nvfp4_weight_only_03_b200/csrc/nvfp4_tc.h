@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "nvfp4_prologue.h"
+
 namespace nvfp4_tc {
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -21,17 +23,19 @@ int choose_splits(int64_t n, int64_t k, int sms);
 size_t scratch_bytes(int64_t n, int64_t k, int m, int sms);
 // The tier's TMA scale boxes need K % 256 == 0 and 16-byte aligned scale codes.
 bool usable(const void* s, int64_t k);
-// Enqueue one call (arguments already checked as for nvfp4_gemv, 9 <= m <= 128).  The error
-// word is the workspace's first int32; the scratch starts scratch_off bytes in.
+// Enqueue one call (arguments already checked as for nvfp4_gemv, 9 <= m <= 128), with x's
+// prologue applied by the pass that makes its f16 copy.  The error word is the workspace's
+// first int32; the scratch starts scratch_off bytes in.
 int launch(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g, const void* x,
-           int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws,
-           size_t ws_bytes, size_t scratch_off, cudaStream_t stream);
+           int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
+           const nvfp4_pro::Prologue& pro, void* ws, size_t ws_bytes, size_t scratch_off,
+           cudaStream_t stream);
 // The fused dual: o = bf16(silu(g_g W_gate x) * (g_u W_up x)), the two streams through the tier
 // into fp32, then one combining pass.
 int launch_dual(EncodeFn encode, int sms, const uint8_t* wg, const uint8_t* sg, float gg,
                 const uint8_t* wu, const uint8_t* su, float gu, const void* x, int64_t ldx,
-                void* y, int64_t ldy, int m, int64_t n, int64_t k, void* ws, size_t ws_bytes,
-                size_t scratch_off, cudaStream_t stream);
+                void* y, int64_t ldy, int m, int64_t n, int64_t k, const nvfp4_pro::Prologue& pro,
+                void* ws, size_t ws_bytes, size_t scratch_off, cudaStream_t stream);
 
 }  // namespace nvfp4_tc
 

@@ -15,6 +15,10 @@ Workload recipes (the projection shapes of a 27B hybrid GatedDeltaNet + gated-at
   sweep     4 layers x {qkv 10240x5120, o 5120x6144, gate_up 2x17408x5120, down 5120x17408},
             M in {1,2,4,8}, seed 4
 
+Input prologues (the residual add + RMS norm before a projection, the sigmoid gate before the
+attention output projection): a residual stream of N(0, 4^2) bf16 draws, norm gains
+1 + N(0, 0.1^2) rounded to bf16, gate logits N(0, 2^2) bf16, each from its own offset.
+
 Stream order inside one seed: every weight tensor (row-major, in the order listed; for the dual,
 gate then up), then every activation tensor (row-major).  Activations are always drawn with 8 rows
 and an M-row call uses the first M, so row r of x is the same for every M.
@@ -152,6 +156,22 @@ def nvfp4_weight(seed: int, offset: int, n: int, k: int, sigma: float = W_SIGMA)
 def activations(seed: int, offset: int, m: int, k: int) -> np.ndarray:
     """bf16 bits [m][k] of N(0, 1) draws."""
     return normal_bf16(seed, offset, m * k, X_SIGMA).reshape(m, k)
+
+
+def residual_stream(seed: int, offset: int, m: int, k: int, sigma: float = 4.0) -> np.ndarray:
+    """bf16 bits [m][k] of N(0, sigma^2) draws: the residual stream a norm prologue adds."""
+    return normal_bf16(seed, offset, m * k, sigma).reshape(m, k)
+
+
+def norm_gains(seed: int, offset: int, k: int, sigma: float = 0.1) -> np.ndarray:
+    """bf16 bits [k] of 1 + N(0, sigma^2): an RMS norm's per-channel gains."""
+    v = normal_f32(seed, offset, k, sigma) + np.float32(1.0)
+    return np.array([f32_to_bf16(float(t)) for t in v], np.uint16)
+
+
+def gate_logits(seed: int, offset: int, m: int, k: int, sigma: float = 2.0) -> np.ndarray:
+    """bf16 bits [m][k] of N(0, sigma^2): the pre-sigmoid gate of a gated output."""
+    return normal_bf16(seed, offset, m * k, sigma).reshape(m, k)
 
 
 # ----------------------------------------------------------------------------------------------

@@ -194,3 +194,88 @@ def test_wide_tensor_flag_host_checks(L):
     assert L.nvfp4_workspace_bytes_wide(64, 64, 129, ctypes.byref(b)) == -3
     if not cuda_ok():
         assert L.nvfp4_workspace_bytes_wide(64, 64, 16, ctypes.byref(b)) == -5
+
+
+# ---- input prologues: host checks (distinct fake addresses so that only the planted overlap
+# counts as one)
+PX, PY, PR, PG, PH, PT, PW, PWS = (0x100000 * i for i in range(1, 9))
+
+
+def pro(kind=nv.PROLOGUE_ADD_RMSNORM, eps=1e-6, residual=PR, ld_residual=64, gamma=PG,
+        residual_out=PH, ld_residual_out=64, gate=PT, ld_gate=64):
+    return nv.Prologue(kind=kind, eps=eps, residual=residual, ld_residual=ld_residual,
+                       gamma=gamma, residual_out=residual_out, ld_residual_out=ld_residual_out,
+                       gate=gate, ld_gate=ld_gate)
+
+
+def call_pro(L, p, m=2, n=64, k=64):
+    return L.nvfp4_gemv_pro(ctypes.byref(p) if p is not None else None, PW, PW, 1.0, PX, k, PY,
+                            n, m, n, k, PWS, 1 << 30, 0, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(kind=7), -2), (dict(kind=-1), -2),
+    (dict(eps=-1.0), -2), (dict(eps=float("nan")), -2), (dict(eps=float("inf")), -2),
+    (dict(residual=None), -1), (dict(gamma=None), -1),
+    (dict(ld_residual=32), -2), (dict(ld_residual_out=32), -2),
+    (dict(ld_residual=68), -4), (dict(residual=PR + 8), -4), (dict(gamma=PG + 8), -4),
+    (dict(residual_out=PH + 8), -4), (dict(ld_residual_out=72 + 4), -4),
+    (dict(residual_out=PX), -8),            # h written over x
+    (dict(residual_out=PR + 64), -8),       # ... over the residual's second row
+    (dict(residual_out=PG - 32), -8),       # ... over gamma
+    (dict(residual_out=PY + 2 * 64), -8),   # ... over y's second row
+    (dict(residual=PY), -8),                # y written over the residual
+    (dict(kind=nv.PROLOGUE_SIGMOID_GATE, gate=None), -1),
+    (dict(kind=nv.PROLOGUE_SIGMOID_GATE, ld_gate=8), -2),
+    (dict(kind=nv.PROLOGUE_SIGMOID_GATE, gate=PT + 2), -4),
+    (dict(kind=nv.PROLOGUE_SIGMOID_GATE, gate=PY), -8),
+])
+def test_prologue_host_checks(L, kw, status):
+    assert call_pro(L, pro(**kw)) == status
+
+
+def test_prologue_valid_calls_and_noops(L):
+    # no prologue or kind NONE is the plain call; a gate prologue ignores the norm fields
+    expect = 0 if cuda_ok() else -5
+    for p in (None, pro(kind=nv.PROLOGUE_NONE, residual=None, gamma=None),
+              pro(), pro(residual_out=None),
+              pro(kind=nv.PROLOGUE_SIGMOID_GATE, residual=None, gamma=None, eps=-5.0)):
+        if not cuda_ok():
+            assert call_pro(L, p) == expect
+    # M == 0: nothing is read; the kind and eps are still checked
+    assert call_pro(L, pro(residual=None, gamma=None), m=0) == 0
+    assert call_pro(L, pro(kind=9), m=0) == -2
+    # the tensors of the prologue stay clear of x where x's rows are strided past K
+    assert call_pro(L, pro(residual_out=PX + 2 * 64 * 2), m=1) == (0 if cuda_ok() else -5)
+
+
+def test_dual_and_multi_prologue_host_checks(L):
+    p = pro(residual_out=PY)
+    st = L.nvfp4_gemv_dual_pro(ctypes.byref(p), PW, PW, 1.0, PW, PW, 1.0, PX, 64, PY, 64, 2, 64,
+                               64, PWS, 1 << 30, 0, None)
+    assert st == -8
+    outs = _outputs((PW, PW, 1.0, PY, 64, 64), (PW, PW, 1.0, PY + 0x10000, 64, 64))
+    p2 = pro(residual_out=PY + 0x10000 + 64)  # overlaps the second output
+    assert L.nvfp4_gemv_multi_pro(ctypes.byref(p2), outs, 2, PX, 64, 2, 64, PWS, 1 << 30, 0,
+                                  None) == -8
+    p3 = pro(kind=3)
+    assert L.nvfp4_gemv_multi_pro(ctypes.byref(p3), outs, 2, PX, 64, 2, 64, PWS, 1 << 30, 0,
+                                  None) == -2
+    if not cuda_ok():
+        p4 = pro()
+        assert L.nvfp4_gemv_multi_pro(ctypes.byref(p4), outs, 2, PX, 64, 2, 64, PWS, 1 << 30, 0,
+                                      None) == -5
+
+
+def test_prologue_binding_argument_checks():
+    import torch
+    w = torch.zeros((64, 32), dtype=torch.uint8)
+    s = torch.zeros((64, 4), dtype=torch.uint8)
+    x = torch.zeros((2, 64), dtype=torch.bfloat16)
+    r = torch.zeros((2, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):  # gamma of the wrong length
+        nv.gemv(w, s, 1.0, x, prologue=nv.AddRmsNorm(r, torch.ones(32, dtype=torch.bfloat16)))
+    with pytest.raises(ValueError):  # residual of the wrong shape
+        nv.gemv(w, s, 1.0, x, prologue=nv.AddRmsNorm(r[:1], torch.ones(64, dtype=torch.bfloat16)))
+    with pytest.raises(TypeError):   # gate not bf16
+        nv.gemv(w, s, 1.0, x, prologue=nv.SigmoidGate(torch.zeros((2, 64))))

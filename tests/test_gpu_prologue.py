@@ -1,0 +1,220 @@
+"""Input prologues through the C ABI against the oracle: residual add + RMS norm (single, dual,
+multi-output, 8-row passes, the tensor-core tier) and the sigmoid gate.
+
+The GPU forms x' in fp32 and rounds it to bf16; the oracle forms it in fp64.  Where the fp64
+value lies within a relative 2^-16 of a bf16 rounding midpoint the two may round apart, so the
+tolerance of each output grows by sum_k |w_k| * (one bf16 step of x'_k) over those elements
+(oracle.rounding_slack); everywhere else the acceptance rules are unchanged.  The residual sum h
+is exactly rounded on both sides and compared bitwise."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import nvfp4_weight_only_03_b200 as nv
+from gpu_util import bits, check_dual, check_single, dev_weight, dev_x
+
+pytestmark = pytest.mark.gpu
+
+
+def dev_vec(v_bits):
+    return torch.from_numpy(np.ascontiguousarray(v_bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def check_pro_single(y_bits, w, xq, near, where, rows=None):
+    ref, a = oracle.gemv(w.packed, w.scales, w.g, xq, rows=rows)
+    _, extra = oracle.gemv(w.packed, w.scales, w.g, oracle.rounding_slack(xq, near), rows=rows)
+    return check_single(y_bits, ref, a + extra / 2e-3, where)
+
+
+def check_pro_dual(o_bits, wg, wu, xq, near, where, rows=None):
+    o_ref, yg, yu, ag, au = oracle.gemv_dual(wg.packed, wg.scales, wg.g, wu.packed, wu.scales,
+                                             wu.g, xq, rows=rows)
+    slack = oracle.rounding_slack(xq, near)
+    _, eg = oracle.gemv(wg.packed, wg.scales, wg.g, slack, rows=rows)
+    _, eu = oracle.gemv(wu.packed, wu.scales, wu.g, slack, rows=rows)
+    return check_dual(o_bits, o_ref, yg, yu, ag + eg / 2e-3, au + eu / 2e-3, where)
+
+
+def norm_inputs(seed, m, k, x_scale=1.0):
+    x = synth.activations(seed, 300_000_000, m, k)
+    r = synth.residual_stream(seed, 310_000_000, m, k)
+    if x_scale != 1.0:  # exact power-of-two scaling of both (bf16 exponent shift)
+        x = oracle.bf16_rne(oracle.bf16_value(x) * x_scale)
+        r = oracle.bf16_rne(oracle.bf16_value(r) * x_scale)
+    gamma = synth.norm_gains(seed, 320_000_000, k)
+    return x, r, gamma
+
+
+def sample_rows(n, count=160):
+    if n <= 2048:
+        return None
+    return np.unique(np.concatenate([np.random.default_rng(n).integers(0, n, count),
+                                     [0, 127, 128, n - 1]]))
+
+
+@pytest.mark.parametrize("m", [1, 8])
+def test_add_rmsnorm_single(m):
+    n, k, eps = 4096 + 77, 5120, 1e-6
+    w = synth.nvfp4_weight(40, 0, n, k)
+    x, r, gamma = norm_inputs(40, m, k)
+    W, S, g = dev_weight(w)
+    h_out = torch.full((m, k), float("nan"), dtype=torch.bfloat16, device="cuda")
+    pro = nv.AddRmsNorm(dev_x(r), dev_vec(gamma), eps, h_out)
+    y = bits(nv.gemv(W, S, g, dev_x(x), prologue=pro))
+    h_ref, xn, near = oracle.add_rmsnorm(x, r, gamma, eps)
+    assert np.array_equal(bits(h_out), h_ref), "residual sum h"
+    rows = sample_rows(n)
+    check_pro_single(y if rows is None else y[:, rows], w, xn, near, f"add_rmsnorm M={m}", rows)
+    # determinism, and each row as in a call of its own
+    assert np.array_equal(bits(nv.gemv(W, S, g, dev_x(x), prologue=pro)), y)
+    for i in (0, m - 1):
+        y1 = bits(nv.gemv(W, S, g, dev_x(x[i:i + 1]),
+                          prologue=nv.AddRmsNorm(dev_x(r[i:i + 1]), dev_vec(gamma), eps)))
+        assert np.array_equal(y1[0], y[i]), f"row {i}"
+
+
+@pytest.mark.parametrize("scale,eps", [(2.0 ** -14, 1e-6), (1.0, 0.5), (2.0 ** 20, 0.0)])
+def test_add_rmsnorm_eps_and_magnitudes(scale, eps):
+    # eps dominating the mean square, a large eps, and large magnitudes with eps = 0
+    n, k, m = 1000, 2048, 3
+    w = synth.nvfp4_weight(41, 0, n, k)
+    x, r, gamma = norm_inputs(41, m, k, x_scale=scale)
+    W, S, g = dev_weight(w)
+    y = bits(nv.gemv(W, S, g, dev_x(x), prologue=nv.AddRmsNorm(dev_x(r), dev_vec(gamma), eps)))
+    _, xn, near = oracle.add_rmsnorm(x, r, gamma, eps)
+    check_pro_single(y, w, xn, near, f"scale={scale} eps={eps}")
+
+
+def test_add_rmsnorm_dual():
+    n, k, m, eps = 2048, 5120, 4, 1e-6
+    wg = synth.nvfp4_weight(42, 0, n, k)
+    wu = synth.nvfp4_weight(42, 20_000_000, n, k)
+    x, r, gamma = norm_inputs(42, m, k)
+    Wg, Sg, gg = dev_weight(wg)
+    Wu, Su, gu = dev_weight(wu)
+    h_out = torch.empty((m, k), dtype=torch.bfloat16, device="cuda")
+    o = bits(nv.gemv_dual(Wg, Sg, gg, Wu, Su, gu, dev_x(x),
+                          prologue=nv.AddRmsNorm(dev_x(r), dev_vec(gamma), eps, h_out)))
+    h_ref, xn, near = oracle.add_rmsnorm(x, r, gamma, eps)
+    assert np.array_equal(bits(h_out), h_ref)
+    check_pro_dual(o, wg, wu, xn, near, "dual add_rmsnorm")
+
+
+def test_add_rmsnorm_multi():
+    # the attention projections sharing the normed x: q (6144) and k, v (1024 each)
+    k, m, eps = 5120, 3, 1e-6
+    ws_ = [synth.nvfp4_weight(43, off, n, k) for off, n in
+           ((0, 6144), (40_000_000, 1024), (50_000_000, 1024))]
+    x, r, gamma = norm_inputs(43, m, k)
+    devs = [dev_weight(w) for w in ws_]
+    h_out = torch.empty((m, k), dtype=torch.bfloat16, device="cuda")
+    ys = [bits(y) for y in nv.gemv_multi(devs, dev_x(x), prologue=nv.AddRmsNorm(
+        dev_x(r), dev_vec(gamma), eps, h_out))]
+    h_ref, xn, near = oracle.add_rmsnorm(x, r, gamma, eps)
+    assert np.array_equal(bits(h_out), h_ref)
+    for o, (w, y) in enumerate(zip(ws_, ys)):
+        rows = sample_rows(w.n)
+        check_pro_single(y if rows is None else y[:, rows], w, xn, near, f"multi output {o}", rows)
+
+
+@pytest.mark.parametrize("m", [1, 8])
+def test_sigmoid_gate_single(m):
+    # the attention output projection: o 5120 x 6144 after the sigmoid gate
+    n, k = 5120, 6144
+    w = synth.nvfp4_weight(44, 0, n, k)
+    a = synth.activations(44, 300_000_000, m, k)
+    t = synth.gate_logits(44, 310_000_000, m, k)
+    W, S, g = dev_weight(w)
+    y = bits(nv.gemv(W, S, g, dev_x(a), prologue=nv.SigmoidGate(dev_x(t))))
+    xo, near = oracle.sigmoid_gate(a, t)
+    rows = sample_rows(n)
+    check_pro_single(y[:, rows], w, xo, near, f"sigmoid gate M={m}", rows)
+    if m > 1:
+        y1 = bits(nv.gemv(W, S, g, dev_x(a[m - 1:]), prologue=nv.SigmoidGate(dev_x(t[m - 1:]))))
+        assert np.array_equal(y1[0], y[m - 1])
+
+
+def test_prologue_with_ragged_k_and_passes():
+    # K % 256 != 0 (partial last unit), 19 rows (three 8-row passes), strided arrays
+    n, k, m, eps = 700, 5120 + 96, 19, 1e-5
+    w = synth.nvfp4_weight(45, 0, n, k)
+    x, r, gamma = norm_inputs(45, m, k)
+    W, S, g = dev_weight(w)
+    hbuf = torch.full((m, k + 40), float("nan"), dtype=torch.bfloat16, device="cuda")
+    pro = nv.AddRmsNorm(dev_x(r, ldx=k + 64), dev_vec(gamma), eps, hbuf[:, :k])
+    y = bits(nv.gemv(W, S, g, dev_x(x, ldx=k + 128), prologue=pro))
+    h_ref, xn, near = oracle.add_rmsnorm(x, r, gamma, eps)
+    assert np.array_equal(bits(hbuf[:, :k]), h_ref)
+    assert torch.isnan(hbuf[:, k:].float()).all(), "wrote past K in residual_out"
+    check_pro_single(y, w, xn, near, "ragged K, 19 rows")
+    for i in (0, 8, 18):
+        y1 = bits(nv.gemv(W, S, g, dev_x(x[i:i + 1]),
+                          prologue=nv.AddRmsNorm(dev_x(r[i:i + 1]), dev_vec(gamma), eps)))
+        assert np.array_equal(y1[0], y[i]), f"row {i}"
+    # a gate prologue at the same ragged K
+    t = synth.gate_logits(45, 330_000_000, m, k)
+    y = bits(nv.gemv(W, S, g, dev_x(x), prologue=nv.SigmoidGate(dev_x(t))))
+    xo, near = oracle.sigmoid_gate(x, t)
+    check_pro_single(y, w, xo, near, "gate, ragged K, 19 rows")
+
+
+def test_kind_none_is_the_plain_call():
+    n, k, m = 1500, 2048, 5
+    w = synth.nvfp4_weight(46, 0, n, k)
+    x = synth.activations(46, 300_000_000, m, k)
+    W, S, g = dev_weight(w)
+
+    class NoneKind:
+        def struct(self, m_, k_):
+            return nv.Prologue(kind=nv.PROLOGUE_NONE)
+
+    assert np.array_equal(bits(nv.gemv(W, S, g, dev_x(x), prologue=NoneKind())),
+                          bits(nv.gemv(W, S, g, dev_x(x))))
+
+
+def test_prologue_on_the_tensor_core_tier():
+    n, k, m, eps = 4096, 5120, 24, 1e-6
+    w = synth.nvfp4_weight(47, 0, n, k)
+    wu = synth.nvfp4_weight(47, 30_000_000, n, k)
+    x, r, gamma = norm_inputs(47, m, k)
+    W, S, g = dev_weight(w)
+    Wu, Su, gu = dev_weight(wu)
+    h_out = torch.empty((m, k), dtype=torch.bfloat16, device="cuda")
+    pro = nv.AddRmsNorm(dev_x(r), dev_vec(gamma), eps, h_out)
+    y = bits(nv.gemv(W, S, g, dev_x(x), prologue=pro, wide_tensor=True))
+    h_ref, xn, near = oracle.add_rmsnorm(x, r, gamma, eps)
+    assert np.array_equal(bits(h_out), h_ref)
+    rows = sample_rows(n)
+    check_pro_single(y[:, rows], w, xn, near, "tier add_rmsnorm", rows)
+    # rows invariant within the tier (9..24 rows)
+    y9 = bits(nv.gemv(W, S, g, dev_x(x[:9]), wide_tensor=True,
+                      prologue=nv.AddRmsNorm(dev_x(r[:9]), dev_vec(gamma), eps)))
+    assert np.array_equal(y9, y[:9])
+    o = bits(nv.gemv_dual(W, S, g, Wu, Su, gu, dev_x(x), wide_tensor=True,
+                          prologue=nv.AddRmsNorm(dev_x(r), dev_vec(gamma), eps)))
+    check_pro_dual(o[:, rows], w, wu, xn, near, "tier dual add_rmsnorm", rows)
+    t = synth.gate_logits(47, 330_000_000, m, k)
+    y = bits(nv.gemv(W, S, g, dev_x(x), prologue=nv.SigmoidGate(dev_x(t)), wide_tensor=True))
+    xo, near = oracle.sigmoid_gate(x, t)
+    check_pro_single(y[:, rows], w, xo, near, "tier sigmoid gate", rows)
+    assert nv.workspace_error(nv.wide_workspace(n, k, m)) == 0
+
+
+def test_prologue_needs_the_larger_workspace():
+    n, k, m = 256, 512, 2
+    w = synth.nvfp4_weight(48, 0, n, k)
+    x, r, gamma = norm_inputs(48, m, k)
+    W, S, g = dev_weight(w)
+    small = torch.zeros(nv.workspace_bytes(), dtype=torch.uint8, device="cuda")
+    assert nv.workspace_bytes_wide(n, k, m) > nv.workspace_bytes()
+    with pytest.raises(nv.Nvfp4Error) as e:
+        nv.gemv(W, S, g, dev_x(x), ws=small,
+                prologue=nv.AddRmsNorm(dev_x(r), dev_vec(gamma), 1e-6))
+    assert e.value.status == -7
+    big = torch.zeros(nv.workspace_bytes_wide(n, k, m), dtype=torch.uint8, device="cuda")
+    y = bits(nv.gemv(W, S, g, dev_x(x), ws=big,
+                     prologue=nv.AddRmsNorm(dev_x(r), dev_vec(gamma), 1e-6)))
+    _, xn, near = oracle.add_rmsnorm(x, r, gamma, 1e-6)
+    check_pro_single(y, w, xn, near, "explicit workspace")
