@@ -273,7 +273,8 @@ int nvfp4_gemv_noalloc(const uint8_t* w, const uint8_t* s, float global_scale, c
                        int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
                        cudaStream_t stream);
 
-/* Workspace bytes of an nvfp4_gemv_ex / _pro or nvfp4_gemv_dual_ex / _pro call of M rows with
+/* Workspace bytes of an nvfp4_gemv_ex / _pro, nvfp4_gemv_dual_ex / _pro or nvfp4_gemv_multi_pro
+ * (N = its largest output) call of M rows with
  * NVFP4_FLAG_WIDE_TENSOR or an input prologue: the nvfp4_workspace_bytes layout followed by the
  * larger of the tier's scratch (fp32 partial sums of its split of K, an f16 copy of x with the
  * rows' scales, and the dual's two fp32 results; the size depends on N, K, M and the SM count)
