@@ -66,12 +66,12 @@ def parse():
 # launch, for layer 0 of the sweep at M = 1 and M = 8 (profiles/nvfp4_gemv_sweep_dram_traffic.md).
 # They describe the kernel code with this SHA-256 only (kernel_code_sha256: comments and blank
 # lines do not count); for any other code the bench reports traffic as null.
-TRAFFIC_SOURCE_SHA256 = "ee6c5010fb162609c1317241ee9af6bd097f7543628b6e1361b6027ffd8ccefa"
+TRAFFIC_SOURCE_SHA256 = "d8dd8c23be2b377cc368e69df00b59b272e467ef9de2bc97e947e3aa55087079"
 TRAFFIC_BYTES = {
-    ("L0.qkv", 1): 30119168, ("L0.o", 1): 18324480, ("L0.gate_up", 1): 106838784,
-    ("L0.down", 1): 50807040,
-    ("L0.qkv", 8): 29617152, ("L0.o", 8): 17837568, ("L0.gate_up", 8): 108867328,
-    ("L0.down", 8): 50468864,
+    ("L0.qkv", 1): 30118912, ("L0.o", 1): 18324480, ("L0.gate_up", 1): 106766592,
+    ("L0.down", 1): 50805248,
+    ("L0.qkv", 8): 29616640, ("L0.o", 8): 17837312, ("L0.gate_up", 8): 106094592,
+    ("L0.down", 8): 50467584,
 }
 KERNEL_SOURCE = os.path.join(ROOT, "nvfp4_weight_only_03_b200", "csrc", "nvfp4_gemv.cu")
 
