@@ -1,17 +1,17 @@
-// Input prologues of the GEMV kernels: the transforms of x that the decode step runs just
-// before a projection, applied while x is staged instead of in launches of their own
-// ("Blueprint - circuit executor" page for qwen3.8-27b-nvfp4 on GB10, table "Kernels the plan
-// launches": residual_add_rms_norm / rms_norm before the attention and FFN projections,
-// sigmoid_gate_mul before the attention output projection).
+// Input prologues of the GEMV calls: the transforms of x that the decode step runs just before
+// a projection ("Blueprint - circuit executor" page for qwen3.8-27b-nvfp4 on GB10, table "Kernels
+// the plan launches": residual_add_rms_norm / rms_norm before the attention and FFN projections,
+// sigmoid_gate_mul before the attention output projection).  The prologue grid ahead of the
+// 1..8-row GEMV (nvfp4_gemv.cu) and the x pass of the tensor-core tier (nvfp4_gemv_tc.cu) both
+// use these helpers, so the two form x' with the same operations.
 //
 //   NVFP4_PROLOGUE_ADD_RMSNORM:  h = bf16(x + r);  x' = bf16((h * inv) * gamma),
 //                                inv = 1 / sqrt(sum_k h^2 / K + eps)
 //   NVFP4_PROLOGUE_SIGMOID_GATE: x' = bf16(x / (1 + e^-gate))
 //
 // in fp32.  x + r of two bf16 values rounded once to bf16 equals the exactly rounded sum (fp32
-// carries more than twice bf16's precision plus two bits).  The sum of squares runs in a fixed
-// order that depends on neither M nor the CTA (see sum_squares_8), so every CTA of a launch,
-// and every M, sees the same inv for a row.
+// carries more than twice bf16's precision plus two bits).  Each caller sums a row's squares in
+// an order fixed by K alone, so x' of a row does not depend on M.
 #ifndef NVFP4_PROLOGUE_H
 #define NVFP4_PROLOGUE_H
 
@@ -31,14 +31,6 @@ struct Prologue {
     uint16_t* hout;        // ADD_RMSNORM: h = bf16(x + r), bf16 [M][ldh], or null
     int64_t ldh;
 };
-
-// The same prologue for rows r0.. of a call (8-row passes).
-inline Prologue rows_from(const Prologue& p, int64_t r0) {
-    Prologue q = p;
-    if (q.in) q.in += r0 * q.ld_in;
-    if (q.hout) q.hout += r0 * q.ldh;
-    return q;
-}
 
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
