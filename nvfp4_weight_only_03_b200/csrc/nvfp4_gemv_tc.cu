@@ -49,8 +49,13 @@ constexpr int kABytes = kRows * kStageK * 2;    // 16384: decoded f16 tile
 #ifndef NVFP4_TC_ABUF
 #define NVFP4_TC_ABUF 2
 #endif
-constexpr int kStages = 6;                  // x tiles in flight (one per 64-k stage)
-constexpr int kUStages = 4;                 // weight units in flight (one per 256 k)
+constexpr int kStages = 6;                  // x tiles in flight at most (one per 64-k stage)
+constexpr int kUStages = 2;                 // weight units in flight (one per 256 k)
+// Two CTAs share an SM: each CTA's stages are bound by its own hand-offs (TMA -> decode -> MMA
+// -> commit), not by a resource the SM's other CTA needs, so a second CTA overlaps them.  Each
+// then has half of the SM's shared memory (228 KB, less 1 KB reserved per CTA).
+constexpr int kCtasPerSm = 2;
+constexpr size_t kCtaSmemBudget = 233472 / kCtasPerSm - 1024;
 constexpr int kABuf = NVFP4_TC_ABUF;        // decoded tiles in flight
 constexpr int kDecodeWarps = 8;             // two threads per weight row
 constexpr int kDecoders = kDecodeWarps * 32;
@@ -59,13 +64,22 @@ constexpr int kMmaWarp = 1 + kDecodeWarps;
 constexpr int kTmemCols = 128;
 constexpr int kSpinLimit = 1 << 24;
 // shared memory: kUStages weight units (nibbles with 128-byte swizzle, then scale codes), kABuf
-// decoded tiles, kStages x tiles (N rows of 128 bytes, 128-byte swizzle); N is a multiple of 16,
-// so every piece keeps the 1024-byte alignment of the swizzle
-constexpr size_t smem_bytes(int nx) {
-    return 1024 + (size_t)kUStages * kUnitBytes + (size_t)kABuf * kABytes +
-           (size_t)kStages * nx * kXRowBytes;
+// decoded tiles, then as many x tiles (N rows of 128 bytes, 128-byte swizzle) as the CTA's
+// share holds, at most kStages; N is a multiple of 16, so every piece keeps the 1024-byte
+// alignment of the swizzle
+__host__ __device__ constexpr size_t fixed_bytes() {
+    return 1024 + (size_t)kUStages * kUnitBytes + (size_t)kABuf * kABytes;
 }
-constexpr size_t kSmemMax = smem_bytes(kMaxXRows);
+__host__ __device__ constexpr int x_stages(int nx) {
+    return (int)((kCtaSmemBudget - fixed_bytes()) / ((size_t)nx * kXRowBytes)) > kStages
+               ? kStages
+               : (int)((kCtaSmemBudget - fixed_bytes()) / ((size_t)nx * kXRowBytes));
+}
+constexpr size_t smem_bytes(int nx) {
+    return fixed_bytes() + (size_t)x_stages(nx) * nx * kXRowBytes;
+}
+constexpr size_t kSmemMax = kCtaSmemBudget;
+static_assert(x_stages(kMaxXRows) >= 2, "the x ring needs two tiles at N = 128");
 
 struct TcParams {
     uint16_t* y;        // bf16 [M][ldy] (written when splits == 1 and yf is null)
@@ -185,7 +199,7 @@ __device__ __forceinline__ uint16_t f2bf(float v) {
     return (uint16_t)u;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     nvfp4_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tx,
                     const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap ts) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -199,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ uint32_t tmem_base;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int xst = x_stages(p.nx);  // x ring depth
     const int tile = blockIdx.x / p.splits, split = blockIdx.x - tile * p.splits;
     const int u_begin = (int)((int64_t)p.units * split / p.splits);
     const int u_end = (int)((int64_t)p.units * (split + 1) / p.splits);
@@ -248,8 +263,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(dst, &tw, (u_begin + u) * (kUnitK / 2), tile * kRows, &ufull_bar[us]);
                     tma_load_2d(dst + kWBytes, &ts, (u_begin + u) * 16, tile * kRows, &ufull_bar[us]);
                 }
-                const int slot = s % kStages;
-                if (s >= kStages && !mbar_wait(&xempty_bar[slot], ((s / kStages) - 1) & 1)) {
+                const int slot = s % xst;
+                if (s >= xst && !mbar_wait(&xempty_bar[slot], ((s / xst) - 1) & 1)) {
                     ok = false;
                     break;
                 }
@@ -263,8 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- MMA issuer
         if (lane == 0) {
             for (int s = 0; s < stages && ok; ++s) {
-                const int slot = s % kStages, buf = s % kABuf;
-                if (!mbar_wait(&xfull_bar[slot], (s / kStages) & 1) ||
+                const int slot = s % xst, buf = s % kABuf;
+                if (!mbar_wait(&xfull_bar[slot], (s / xst) & 1) ||
                     !mbar_wait(&afull_bar[buf], (s / kABuf) & 1)) {
                     ok = false;
                     break;
@@ -493,16 +508,17 @@ namespace nvfp4_tc {
 #ifndef NVFP4_TC_ITEM_COST
 #define NVFP4_TC_ITEM_COST 2
 #endif
-// splits: the fewest that minimise the makespan: the waves a CTA runs (ceil(items / sms)) times
-// the cost of an item, its units plus a fixed cost of NVFP4_TC_ITEM_COST units (start-up, the
-// pipeline's fill and drain, writing the partials).  Depends only on (N, K, SM count).
+// splits: the fewest that minimise the makespan: the waves a CTA runs (ceil(items / (2 sms)),
+// two CTAs per SM) times the cost of an item, its units plus a fixed cost of NVFP4_TC_ITEM_COST
+// units (start-up, the pipeline's fill and drain, writing the partials).  Depends only on (N, K,
+// SM count).
 int choose_splits(int64_t n, int64_t k, int sms) {
     const int64_t tiles = (n + kRows - 1) / kRows;
     const int64_t units = (k + kUnitK - 1) / kUnitK;
     int best = 1;
     int64_t best_cost = -1;
     for (int s = 1; s <= 32 && s <= units; ++s) {
-        const int64_t waves = (tiles * s + sms - 1) / sms;
+        const int64_t waves = (tiles * s + kCtasPerSm * sms - 1) / (kCtasPerSm * sms);
         const int64_t per = (units + s - 1) / s;
         const int64_t cost = waves * (per + NVFP4_TC_ITEM_COST);
         if (best_cost < 0 || cost < best_cost) {
@@ -552,8 +568,11 @@ static int set_attr() {
         return NVFP4_ERR_ARCH;
     }
     if (!attr_set[dev]) {
+        // the whole shared-memory carveout, so that two CTAs' shares fit on an SM
         if (cudaFuncSetAttribute(nvfp4_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kSmemMax) != cudaSuccess) {
+                                 (int)kSmemMax) != cudaSuccess ||
+            cudaFuncSetAttribute(nvfp4_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 100) != cudaSuccess) {
             cudaGetLastError();
             return NVFP4_ERR_LAUNCH;
         }
