@@ -218,3 +218,25 @@ def test_prologue_needs_the_larger_workspace():
                      prologue=nv.AddRmsNorm(dev_x(r), dev_vec(gamma), 1e-6)))
     _, xn, near = oracle.add_rmsnorm(x, r, gamma, 1e-6)
     check_pro_single(y, w, xn, near, "explicit workspace")
+
+
+def test_prologue_beyond_one_register_round():
+    # K = 17408 > 4 x 512 chunks of 8: the norm re-reads x, the residual and gamma for x', and
+    # the gate walks its row in several rounds; 12 rows run as two 8-row GEMV passes
+    n, k, m, eps = 640, 17408, 12, 1e-6
+    w = synth.nvfp4_weight(49, 0, n, k)
+    x, r, gamma = norm_inputs(49, m, k)
+    W, S, g = dev_weight(w)
+    h_out = torch.empty((m, k), dtype=torch.bfloat16, device="cuda")
+    y = bits(nv.gemv(W, S, g, dev_x(x), prologue=nv.AddRmsNorm(dev_x(r), dev_vec(gamma), eps,
+                                                                h_out)))
+    h_ref, xn, near = oracle.add_rmsnorm(x, r, gamma, eps)
+    assert np.array_equal(bits(h_out), h_ref)
+    check_pro_single(y, w, xn, near, "norm, K = 17408")
+    y1 = bits(nv.gemv(W, S, g, dev_x(x[5:6]),
+                      prologue=nv.AddRmsNorm(dev_x(r[5:6]), dev_vec(gamma), eps)))
+    assert np.array_equal(y1[0], y[5])
+    t = synth.gate_logits(49, 330_000_000, m, k)
+    y = bits(nv.gemv(W, S, g, dev_x(x), prologue=nv.SigmoidGate(dev_x(t))))
+    xo, near = oracle.sigmoid_gate(x, t)
+    check_pro_single(y, w, xo, near, "gate, K = 17408")
