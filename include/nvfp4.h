@@ -85,14 +85,17 @@ typedef enum {
  *   that earlier work has completed.  Use it only when earlier work on the stream does not
  *   write the weights or scales of this call. */
 #define NVFP4_FLAG_PREFETCH_WEIGHTS 1u
-/* NVFP4_FLAG_WIDE_TENSOR: calls of 9..128 rows with K % 256 == 0 and 16-byte aligned scale
- *   codes run on the tensor-core tier instead of 8-row passes: one pass over each weight,
- *   tcgen05 MMAs on f16 operands (x carried with a power-of-two scale per row) with fp32
- *   accumulation in tensor memory.  For nvfp4_gemv_dual_ex the gate and up results are kept in
- *   fp32 and combined by a final pass, o = bf16(silu(g_gate gate) * (g_up up)).  Rows are then
- *   bitwise invariant for every M in 9..128 and deterministic, and agree with calls of 1..8
- *   rows within the stated tolerance (not bitwise).  The workspace must hold
- *   nvfp4_workspace_bytes_wide(N, K, M) bytes.  Other calls ignore the flag. */
+/* NVFP4_FLAG_WIDE_TENSOR (nvfp4_gemv_ex, nvfp4_gemv_dual_ex, nvfp4_gemv_multi and their _pro
+ *   forms): calls of 9..128 rows with K % 256 == 0 and 16-byte aligned scale codes (every
+ *   output's, for nvfp4_gemv_multi) run on the tensor-core tier instead of 8-row passes: one
+ *   pass over each weight, tcgen05 MMAs on f16 operands (x carried with a power-of-two scale
+ *   per row) with fp32 accumulation in tensor memory.  For nvfp4_gemv_dual_ex the gate and up
+ *   results are kept in fp32 and combined by a final pass, o = bf16(silu(g_gate gate) *
+ *   (g_up up)).  For nvfp4_gemv_multi x is converted once and each output is bitwise that of
+ *   its own nvfp4_gemv_ex call with the flag.  Rows are then bitwise invariant for every M in
+ *   9..128 and deterministic, and agree with calls of 1..8 rows within the stated tolerance
+ *   (not bitwise).  The workspace must hold nvfp4_workspace_bytes_wide(N, K, M) bytes (for
+ *   nvfp4_gemv_multi, the largest over its outputs).  Other calls ignore the flag. */
 #define NVFP4_FLAG_WIDE_TENSOR 2u
 
 typedef struct {
@@ -273,8 +276,8 @@ int nvfp4_gemv_noalloc(const uint8_t* w, const uint8_t* s, float global_scale, c
                        int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
                        cudaStream_t stream);
 
-/* Workspace bytes of an nvfp4_gemv_ex / _pro, nvfp4_gemv_dual_ex / _pro or nvfp4_gemv_multi_pro
- * (N = its largest output) call of M rows with
+/* Workspace bytes of an nvfp4_gemv_ex / _pro, nvfp4_gemv_dual_ex / _pro or nvfp4_gemv_multi /
+ * _pro (the largest of its outputs' sizes) call of M rows with
  * NVFP4_FLAG_WIDE_TENSOR or an input prologue: the nvfp4_workspace_bytes layout followed by the
  * larger of the tier's scratch (fp32 partial sums of its split of K, an f16 copy of x with the
  * rows' scales, and the dual's two fp32 results; the size depends on N, K, M and the SM count)

@@ -327,11 +327,12 @@ def gemv_dual(wg: torch.Tensor, sg: torch.Tensor, gg: float, wu: torch.Tensor, s
 
 
 def gemv_multi(weights, x: torch.Tensor, ys=None, ws: torch.Tensor = None, stream=None,
-               prefetch_weights: bool = False, prologue=None) -> list:
+               prefetch_weights: bool = False, prologue=None, wide_tensor: bool = False) -> list:
     """Several GEMVs sharing x in one pass (nvfp4_gemv_multi): weights is a list of up to
     MAX_OUTPUTS (w, s, g) triples with the same K; returns [y_0, y_1, ...], y_o the GEMV of
     weight o as gemv computes it.  ys: optional preallocated outputs, one per weight.
-    prologue: as for gemv, applied once to the shared x."""
+    prologue: as for gemv, applied once to the shared x.  wide_tensor: 9..128 rows on the
+    tensor-core tier, each output bitwise as gemv(..., wide_tensor=True) computes it."""
     weights = list(weights)
     if not 1 <= len(weights) <= MAX_OUTPUTS:
         raise ValueError(f"1..{MAX_OUTPUTS} weights, got {len(weights)}")
@@ -352,9 +353,13 @@ def gemv_multi(weights, x: torch.Tensor, ys=None, ws: torch.Tensor = None, strea
         outs[o].w, outs[o].s, outs[o].global_scale = w.data_ptr(), s.data_ptr(), float(g)
         outs[o].y, outs[o].ldy, outs[o].n = y.data_ptr(), ldy, n
     if ws is None:
-        ws = wide_workspace(max(n for n, _ in shapes), k, m, x.device) if pro else \
-            workspace(x.device)
-    flags = FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0
+        if pro is not None or wide_tensor:
+            ws = wide_workspace(max(shapes, key=lambda nk: workspace_bytes_wide(nk[0], k, m))[0],
+                                k, m, x.device)
+        else:
+            ws = workspace(x.device)
+    flags = (FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0) | \
+        (FLAG_WIDE_TENSOR if wide_tensor else 0)
     args = (outs, len(weights), x.data_ptr(), ldx, m, k, ws.data_ptr(), ws.numel(), flags,
             _stream(stream))
     if pro is None:

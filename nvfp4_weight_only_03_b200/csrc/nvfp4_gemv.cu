@@ -1432,6 +1432,30 @@ int nvfp4_gemv_multi_pro(const nvfp4_prologue_t* prologue, const nvfp4_output_t*
     DeviceInfo* di = nullptr;
     st = device_info(&dev, &di);
     if (st != NVFP4_OK) return st;
+    if ((flags & NVFP4_FLAG_WIDE_TENSOR) && m > NVFP4_PASS_ROWS && k > 0) {
+        bool all = true;
+        for (int o = 0; o < used; ++o) all = all && nvfp4_tc::usable(sp[o].s[0], k);
+        if (all) {
+            const uint8_t* tw[kMaxOutputs];
+            const uint8_t* ts[kMaxOutputs];
+            float tg[kMaxOutputs];
+            void* ty[kMaxOutputs];
+            int64_t tldy[kMaxOutputs], tn[kMaxOutputs];
+            for (int o = 0; o < used; ++o) {
+                tw[o] = sp[o].w[0];
+                ts[o] = sp[o].s[0];
+                tg[o] = sp[o].g[0];
+                ty[o] = sp[o].y;
+                tldy[o] = sp[o].ldy;
+                tn[o] = sp[o].n;
+            }
+            size_t flags_off, partial_off;
+            const size_t base = workspace_layout(di->sms, &flags_off, &partial_off);
+            return nvfp4_tc::launch_multi(g_encode, di->sms, tw, ts, tg, ty, tldy, tn, used, x,
+                                          ldx, m, k, pro, workspace, workspace_bytes, base,
+                                          stream);
+        }
+    }
     if ((st = prologue_pass(pro, &x, &ldx, m, k, workspace, workspace_bytes, flags, stream)) !=
         NVFP4_OK)
         return st;

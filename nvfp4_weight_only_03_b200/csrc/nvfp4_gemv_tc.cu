@@ -537,12 +537,17 @@ struct Scratch {
     size_t partial, x16, descale, gate, up, total;
 };
 
-static Scratch scratch_layout(int64_t n, int64_t k, int m, int sms, bool dual) {
+// fp32 partial tiles of one weight's call when its K is split
+static size_t partial_bytes(int64_t n, int64_t k, int m, int sms) {
     const int64_t tiles = (n + kRows - 1) / kRows;
     const int splits = choose_splits(n, k, sms);
+    return splits > 1 ? (size_t)tiles * splits * m * kRows * sizeof(float) : 0;
+}
+
+static Scratch scratch_layout(int64_t n, int64_t k, int m, int sms, bool dual) {
     Scratch sc;
     sc.partial = 0;
-    const size_t partial = splits > 1 ? (size_t)tiles * splits * m * kRows * sizeof(float) : 0;
+    const size_t partial = partial_bytes(n, k, m, sms);
     sc.x16 = align256(partial);
     sc.descale = sc.x16 + align256((size_t)m * k * 2);
     sc.gate = sc.descale + align256((size_t)m * sizeof(float));
@@ -701,6 +706,36 @@ int launch_dual(EncodeFn encode, int sms, const uint8_t* wg, const uint8_t* sg, 
     nvfp4_tc_silu_mul<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(
         gate, up, static_cast<uint16_t*>(y), ldy, n, m, gg, gu);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
+    return NVFP4_OK;
+}
+
+int launch_multi(EncodeFn encode, int sms, const uint8_t* const* w, const uint8_t* const* s,
+                 const float* g, void* const* y, const int64_t* ldy, const int64_t* n, int count,
+                 const void* x, int64_t ldx, int m, int64_t k, const nvfp4_pro::Prologue& pro,
+                 void* ws, size_t ws_bytes, size_t scratch_off, cudaStream_t stream) {
+    // one f16 copy of x for every output, after the partial tiles of the largest split
+    size_t need = 0, pmax = 0;
+    for (int o = 0; o < count; ++o) {
+        const size_t b = scratch_bytes(n[o], k, m, sms), pb = partial_bytes(n[o], k, m, sms);
+        need = b > need ? b : need;
+        pmax = pb > pmax ? pb : pmax;
+    }
+    if (ws_bytes < scratch_off + need) return NVFP4_ERR_WORKSPACE;
+    int st = set_attr();
+    if (st != NVFP4_OK) return st;
+    char* const base = static_cast<char*>(ws) + scratch_off;
+    float* const partial = reinterpret_cast<float*>(base);
+    uint16_t* const x16 = reinterpret_cast<uint16_t*>(base + align256(pmax));
+    float* const descale =
+        reinterpret_cast<float*>(base + align256(pmax) + align256((size_t)m * k * 2));
+    nvfp4_tc_prep<<<m, 512, 0, stream>>>(static_cast<const uint16_t*>(x), ldx, k, x16, descale,
+                                         pro);
+    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
+    for (int o = 0; o < count; ++o)
+        if ((st = enqueue_weight(encode, sms, w[o], s[o], g[o], x16, descale, partial, m, n[o], k,
+                                 static_cast<uint16_t*>(y[o]), ldy[o], nullptr,
+                                 static_cast<int32_t*>(ws), stream)) != NVFP4_OK)
+            return st;
     return NVFP4_OK;
 }
 

@@ -37,6 +37,14 @@ int launch_dual(EncodeFn encode, int sms, const uint8_t* wg, const uint8_t* sg, 
                 void* y, int64_t ldy, int m, int64_t n, int64_t k, const nvfp4_pro::Prologue& pro,
                 void* ws, size_t ws_bytes, size_t scratch_off, cudaStream_t stream);
 
+// Several weights sharing x (nvfp4_gemv_multi): one x pass, then each weight through the tier
+// as launch does it, so each output is bitwise that of its own launch.  The workspace must hold
+// the largest scratch_bytes of the outputs.
+int launch_multi(EncodeFn encode, int sms, const uint8_t* const* w, const uint8_t* const* s,
+                 const float* g, void* const* y, const int64_t* ldy, const int64_t* n, int count,
+                 const void* x, int64_t ldx, int m, int64_t k, const nvfp4_pro::Prologue& pro,
+                 void* ws, size_t ws_bytes, size_t scratch_off, cudaStream_t stream);
+
 }  // namespace nvfp4_tc
 
 #endif

@@ -151,3 +151,31 @@ def test_dual_tier_strided_and_fallback():
     # 1..8 rows ignore the flag (bitwise the fused dual kernel)
     o8 = wide_dual(Wg, Sg, gg, Wu, Su, gu, dev_x(x[:8]))
     assert np.array_equal(o8, bits(nv.gemv_dual(Wg, Sg, gg, Wu, Su, gu, dev_x(x[:8]))))
+
+
+def test_multi_on_the_tier_matches_single_calls_and_oracle():
+    # the attention's q and gate (6144 x 5120 each) and k, v (1024 x 5120) sharing x at M = 24
+    k, m = 5120, 24
+    ws_ = [synth.nvfp4_weight(37, off, n, k) for off, n in
+           ((0, 6144), (40_000_000, 1024), (50_000_000, 1024))]
+    x = synth.activations(37, 80_000_000, m, k)
+    devs = [dev_weight(w) for w in ws_]
+    ys = [bits(y) for y in nv.gemv_multi(devs, dev_x(x), wide_tensor=True)]
+    torch.cuda.synchronize()
+    for o, (w, d) in enumerate(zip(ws_, devs)):
+        assert np.array_equal(ys[o], wide(*d, dev_x(x))), f"output {o} vs its own call"
+        rows = np.unique(np.concatenate([np.random.default_rng(o).integers(0, w.n, 120),
+                                         [0, 127, w.n - 1]]))
+        ref, a = oracle.gemv(w.packed, w.scales, w.g, x, rows=rows)
+        check_single(ys[o][:, rows], ref, a, f"multi tier output {o}")
+    # rows invariant over M within the tier
+    ys9 = [bits(y) for y in nv.gemv_multi(devs, dev_x(x[:9]), wide_tensor=True)]
+    torch.cuda.synchronize()
+    for o in range(3):
+        assert np.array_equal(ys9[o], ys[o][:9])
+    # 1..8 rows ignore the flag
+    y8 = [bits(y) for y in nv.gemv_multi(devs, dev_x(x[:8]), wide_tensor=True)]
+    p8 = [bits(y) for y in nv.gemv_multi(devs, dev_x(x[:8]))]
+    torch.cuda.synchronize()
+    for o in range(3):
+        assert np.array_equal(y8[o], p8[o])
