@@ -66,12 +66,12 @@ def parse():
 # launch, for layer 0 of the sweep at M = 1 and M = 8 (profiles/nvfp4_gemv_sweep_dram_traffic.md).
 # They describe the kernel code with this SHA-256 only (kernel_code_sha256: comments and blank
 # lines do not count); for any other code the bench reports traffic as null.
-TRAFFIC_SOURCE_SHA256 = "d8dd8c23be2b377cc368e69df00b59b272e467ef9de2bc97e947e3aa55087079"
+TRAFFIC_SOURCE_SHA256 = "f93c361d24e4656960e8b9966fe0f77a3dcce9c44015611b0fc567fe4d7ca6f8"
 TRAFFIC_BYTES = {
-    ("L0.qkv", 1): 30118912, ("L0.o", 1): 18324480, ("L0.gate_up", 1): 106766592,
-    ("L0.down", 1): 50805248,
-    ("L0.qkv", 8): 29616640, ("L0.o", 8): 17837312, ("L0.gate_up", 8): 106094592,
-    ("L0.down", 8): 50467584,
+    ("L0.qkv", 1): 30119168, ("L0.o", 1): 18323968, ("L0.gate_up", 1): 107118848,
+    ("L0.down", 1): 50808320,
+    ("L0.qkv", 8): 29617408, ("L0.o", 8): 17837312, ("L0.gate_up", 8): 105671168,
+    ("L0.down", 8): 50468608,
 }
 KERNEL_SOURCE = os.path.join(ROOT, "nvfp4_weight_only_03_b200", "csrc", "nvfp4_gemv.cu")
 
