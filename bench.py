@@ -1186,9 +1186,33 @@ def run_wide(args, world, rank, local):
     ws = torch.zeros(max(nv.workspace_bytes_wide(e["p"].n, e["p"].k, WIDE_ROWS[-1]) for e in ents),
                      dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
+    if args.profile_steps:
+        # eager steps of the tier at the largest row count, for ncu launch lists
+        m = WIDE_ROWS[-1]
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 3) + args.profile_steps):
+                for e in ents:
+                    p = e["p"]
+                    if p.dual:
+                        st = L.nvfp4_gemv_dual_ex(e["W"].data_ptr(), e["S"].data_ptr(),
+                                                  ctypes.c_float(p.w.g), e["Wu"].data_ptr(),
+                                                  e["Su"].data_ptr(), ctypes.c_float(p.w_up.g),
+                                                  e["x"].data_ptr(), p.k, e["y"].data_ptr(), p.n,
+                                                  m, p.n, p.k, ws.data_ptr(), ws.numel(),
+                                                  nv.FLAG_WIDE_TENSOR, stream.cuda_stream)
+                    else:
+                        st = L.nvfp4_gemv_ex(e["W"].data_ptr(), e["S"].data_ptr(),
+                                             ctypes.c_float(p.w.g), e["x"].data_ptr(), p.k,
+                                             e["y"].data_ptr(), p.n, m, p.n, p.k, ws.data_ptr(),
+                                             ws.numel(), nv.FLAG_WIDE_TENSOR, stream.cuda_stream)
+                    if st != 0:
+                        raise RuntimeError(f"launch failed: {nv.STATUS.get(st, st)}")
+        stream.synchronize()
+        return None
     per_mode = {}
     for mode, flags in (("passes", nv.FLAG_PREFETCH_WEIGHTS), ("tensor_tier", nv.FLAG_WIDE_TENSOR)):
-        per_mode[mode] = run_wide_mode(args, world, L, ents, ws, stream, flags)
+        per_mode[mode] = run_wide_mode(args, world, L, ents, ws, stream, flags,
+                                       ClockSampler(local) if mode == "tensor_tier" else None)
     peak, peak_src = peaks()
     top = per_mode["tensor_tier"][WIDE_ROWS[-1]]
     return {"metric": METRIC, "value": top["GBps"], "unit": "GB/s", "n_gpus": world,
@@ -1203,7 +1227,10 @@ def run_wide(args, world, rank, local):
                          "traffic": None, "peak_source": peaks_bf16()[1],
                          "note": "f16 tcgen05 MMAs against the measured bf16 cuBLAS burst peak "
                                  "(the same rate for f16); the dual runs both streams on the tier"},
-            "per_rows": per_mode, "gpu_launches": None}
+            "per_rows": per_mode,
+            "gpu_launches": (top["kernels_per_step"] * top["steps"]
+                             if top.get("kernels_per_step") is not None else None),
+            "clocks": top.get("clocks")}
 
 
 def peaks_bf16():
@@ -1214,7 +1241,26 @@ def peaks_bf16():
         return 1590.0, "fallback"
 
 
-def run_wide_mode(args, world, L, ents, ws, stream, flags):
+def graph_kernel_nodes(g):
+    """Kernel nodes of a captured CUDA graph (captured with keep_graph=True), or None."""
+    try:
+        from cuda.bindings import runtime as cr
+        graph = g.raw_cuda_graph()
+        if isinstance(graph, int):
+            graph = cr.cudaGraph_t(init_value=graph)
+        err, _, count = cr.cudaGraphGetNodes(graph, 0)
+        err, nodes, count = cr.cudaGraphGetNodes(graph, count)
+        kernels = 0
+        for node in nodes[:count]:
+            err, kind = cr.cudaGraphNodeGetType(node)
+            if kind == cr.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                kernels += 1
+        return kernels
+    except Exception:
+        return None
+
+
+def run_wide_mode(args, world, L, ents, ws, stream, flags, clocks=None):
     import torch
     import nvfp4_weight_only_03_b200 as nv
     per_m = {}
@@ -1237,12 +1283,17 @@ def run_wide_mode(args, world, L, ents, ws, stream, flags):
             for _ in range(max(args.warmup, 3)):
                 launches(stream.cuda_stream)
         stream.synchronize()
-        g = torch.cuda.CUDAGraph()
+        g = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(g, stream=stream):
             launches(torch.cuda.current_stream().cuda_stream)
+        g.instantiate()
+        kernels = graph_kernel_nodes(g)
         g.replay()
         torch.cuda.synchronize()
         steps = max(1, args.steps // m)
+        if clocks is not None and m == WIDE_ROWS[-1]:
+            clocks.start()
+            time.sleep(0.3)
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world)
         torch.cuda.synchronize()
@@ -1254,11 +1305,15 @@ def run_wide_mode(args, world, L, ents, ws, stream, flags):
         torch.cuda.synchronize()
         barrier(world)
         ms = max_over_ranks(t0.elapsed_time(t1), world) / steps
+        clk = clocks.stop() if clocks is not None and m == WIDE_ROWS[-1] else None
         b = sum((2 if e["p"].dual else 1) * (e["p"].n * e["p"].k * 9 // 16) + m * e["p"].k * 2
                 + m * e["p"].n * 2 for e in ents)
         fl = sum((2 if e["p"].dual else 1) * 2 * m * e["p"].n * e["p"].k for e in ents)
         per_m[m] = {"ms_per_step": round(ms, 5), "GBps": round(world * b / (ms * 1e-3) / 1e9, 1),
-                    "TFLOPs": round(world * fl / (ms * 1e-3) / 1e12, 1), "steps": steps}
+                    "TFLOPs": round(world * fl / (ms * 1e-3) / 1e12, 1), "steps": steps,
+                    "kernels_per_step": kernels}
+        if clk is not None:
+            per_m[m]["clocks"] = clk
         del g
     return per_m
 

@@ -10,7 +10,8 @@
 // * Work: a tile is 128 weight rows; K is cut into `splits` equal ranges of 256-k units, and
 //   each CTA computes one (tile, split) item.  The split depends only on (N, K, SM count).
 //   With one split the CTA writes y; otherwise it writes fp32 partials to the workspace and
-//   nvfp4_tc_reduce adds the splits in order.  Deterministic, no atomics.
+//   nvfp4_tc_reduce adds the splits in order (the dual: nvfp4_tc_dual_finish, over both
+//   streams).  Deterministic, no atomics.
 // * Per 64-k stage a producer warp loads, with TMA (no multicast): the x tile (128 rows x 64 k
 //   of bf16, 128-byte swizzle: the MMA's K-major B layout; rows >= M read as zero), the 128
 //   weight rows' packed nibbles (32 bytes each) and the 256-k unit's scale codes.
@@ -82,9 +83,8 @@ constexpr size_t kSmemMax = kCtaSmemBudget;
 static_assert(x_stages(kMaxXRows) >= 2, "the x ring needs two tiles at N = 128");
 
 struct TcParams {
-    uint16_t* y;        // bf16 [M][ldy] (written when splits == 1 and yf is null)
+    uint16_t* y;        // bf16 [M][ldy] when splits == 1; null: fp32 partial tiles instead
     int64_t ldy;
-    float* yf;          // or fp32 [M][n], without g (the dual's two streams)
     int64_t n, k;
     int m;
     int nx;             // MMA N: M rounded up to 16
@@ -362,13 +362,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
                     if (n < p.n) {
                         const int cols = p.m - c0 < 32 ? p.m - c0 : 32;
-                        if (p.splits == 1 && p.yf) {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (j < cols)
-                                    p.yf[(int64_t)(c0 + j) * p.n + n] =
-                                        __uint_as_float(v[j]) * p.descale[c0 + j];
-                        } else if (p.splits == 1) {
+                        if (p.splits == 1 && p.y) {
 #pragma unroll
                             for (int j = 0; j < 32; ++j)
                                 if (j < cols)
@@ -393,33 +387,68 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                      "r"(kTmemCols));
 }
 
-// y[m][n] = bf16(g * 2^-e(m) * sum over splits, in split order, of the partials), or into yf
-// the fp32 2^-e(m) * sum
-__global__ void nvfp4_tc_reduce(const float* __restrict__ partial, const float* __restrict__ descale,
-                                uint16_t* y, int64_t ldy, float* yf, int64_t n, int m, float g,
-                                int splits) {
-    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t total = (int64_t)m * n;
-    if (idx >= total) return;
-    const int mm = (int)(idx / n);
-    const int64_t nn = idx - (int64_t)mm * n;
-    const int64_t tile = nn / kRows, r = nn - tile * kRows;
-    float acc = 0.f;
-    for (int s = 0; s < splits; ++s)
-        acc += partial[(((tile * splits + s) * (int64_t)m) + mm) * kRows + r];
-    if (yf) yf[(int64_t)mm * n + nn] = acc * descale[mm];
-    else y[(int64_t)mm * ldy + nn] = f2bf(acc * descale[mm] * g);
+// The partial tiles of a K split, added in split order: element (m, n) of tile t, split j is
+// partial[((t splits + j) M + m) 128 + n % 128].  Grid: blockIdx.y = row m of x, 4 consecutive
+// outputs per thread (float4 loads; a tile is 128 outputs, so the 4 share a tile).
+
+constexpr int kReduceThreads = 256;
+
+// y[m][n] = bf16(g * 2^-e(m) * sum of the partials)
+__global__ void __launch_bounds__(kReduceThreads)
+    nvfp4_tc_reduce(const float* __restrict__ partial, const float* __restrict__ descale,
+                    uint16_t* y, int64_t ldy, int64_t n, int m, float g, int splits) {
+    const int mm = blockIdx.y;
+    const int64_t n0 = ((int64_t)blockIdx.x * kReduceThreads + threadIdx.x) * 4;
+    if (n0 >= n) return;
+    const int64_t tile = n0 / kRows;
+    const int r = (int)(n0 - tile * kRows);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < splits; ++j) {
+        const float4 v = *reinterpret_cast<const float4*>(
+            partial + (((tile * splits + j) * (int64_t)m) + mm) * kRows + r);
+        acc[0] += v.x;
+        acc[1] += v.y;
+        acc[2] += v.z;
+        acc[3] += v.w;
+    }
+    const float ds = descale[mm];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        if (n0 + i < n) y[(int64_t)mm * ldy + n0 + i] = f2bf(acc[i] * ds * g);
 }
 
-// o[m][n] = bf16(silu(g_g gate) * (g_u up)), silu(t) = t / (1 + e^-t), in fp32
-__global__ void nvfp4_tc_silu_mul(const float* __restrict__ gate, const float* __restrict__ up,
-                                  uint16_t* y, int64_t ldy, int64_t n, int m, float gg, float gu) {
-    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= (int64_t)m * n) return;
-    const int mm = (int)(idx / n);
-    const int64_t nn = idx - (int64_t)mm * n;
-    const float a = gate[idx] * gg, b = up[idx] * gu;
-    y[(int64_t)mm * ldy + nn] = f2bf(a / (1.0f + expf(-a)) * b);
+// The dual's last pass over both streams' partials:
+//   o[m][n] = bf16(silu(g_g 2^-e(m) gate) * (g_u 2^-e(m) up)),  silu(t) = t / (1 + e^-t), fp32
+__global__ void __launch_bounds__(kReduceThreads)
+    nvfp4_tc_dual_finish(const float* __restrict__ pg, const float* __restrict__ pu,
+                         const float* __restrict__ descale, uint16_t* y, int64_t ldy, int64_t n,
+                         int m, float gg, float gu, int splits) {
+    const int mm = blockIdx.y;
+    const int64_t n0 = ((int64_t)blockIdx.x * kReduceThreads + threadIdx.x) * 4;
+    if (n0 >= n) return;
+    const int64_t tile = n0 / kRows;
+    const int r = (int)(n0 - tile * kRows);
+    float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < splits; ++j) {
+        const int64_t off = (((tile * splits + j) * (int64_t)m) + mm) * kRows + r;
+        const float4 a = *reinterpret_cast<const float4*>(pg + off);
+        const float4 b = *reinterpret_cast<const float4*>(pu + off);
+        ag[0] += a.x;
+        ag[1] += a.y;
+        ag[2] += a.z;
+        ag[3] += a.w;
+        au[0] += b.x;
+        au[1] += b.y;
+        au[2] += b.z;
+        au[3] += b.w;
+    }
+    const float ds = descale[mm];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        if (n0 + i < n) {
+            const float a = ag[i] * ds * gg, b = au[i] * ds * gu;
+            y[(int64_t)mm * ldy + n0 + i] = f2bf(a / (1.0f + expf(-a)) * b);
+        }
 }
 
 // The f16 copy of x (after the call's prologue, if any): row m scaled by 2^e(m) so that its
@@ -531,29 +560,28 @@ int choose_splits(int64_t n, int64_t k, int sms) {
 
 static size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
-// Scratch of a call: fp32 partials (when K is split), the f16 copy of x, the row descales, and
-// for the dual the two streams' fp32 results.
-struct Scratch {
-    size_t partial, x16, descale, gate, up, total;
-};
-
-// fp32 partial tiles of one weight's call when its K is split
-static size_t partial_bytes(int64_t n, int64_t k, int m, int sms) {
+// fp32 partial tiles of one weight's call: when its K is split, and always for the dual's
+// streams (their last pass reads both)
+static size_t partial_bytes(int64_t n, int64_t k, int m, int sms, bool always = false) {
     const int64_t tiles = (n + kRows - 1) / kRows;
     const int splits = choose_splits(n, k, sms);
-    return splits > 1 ? (size_t)tiles * splits * m * kRows * sizeof(float) : 0;
+    return (splits > 1 || always) ? (size_t)tiles * splits * m * kRows * sizeof(float) : 0;
 }
+
+// Scratch of a call: fp32 partial tiles (the dual: one set per stream), the f16 copy of x and
+// the row descales.
+struct Scratch {
+    size_t partial, partial_up, x16, descale, total;
+};
 
 static Scratch scratch_layout(int64_t n, int64_t k, int m, int sms, bool dual) {
     Scratch sc;
+    const size_t pb = align256(partial_bytes(n, k, m, sms, dual));
     sc.partial = 0;
-    const size_t partial = partial_bytes(n, k, m, sms);
-    sc.x16 = align256(partial);
+    sc.partial_up = pb;
+    sc.x16 = dual ? 2 * pb : pb;
     sc.descale = sc.x16 + align256((size_t)m * k * 2);
-    sc.gate = sc.descale + align256((size_t)m * sizeof(float));
-    const size_t res = dual ? align256((size_t)m * n * sizeof(float)) : 0;
-    sc.up = sc.gate + res;
-    sc.total = sc.up + res;
+    sc.total = sc.descale + align256((size_t)m * sizeof(float));
     return sc;
 }
 
@@ -589,7 +617,7 @@ static int set_attr() {
 // The weight's tile pass over the f16 copy of x (already written), then the split reduction.
 static int enqueue_weight(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g,
                           const uint16_t* x16, const float* descale, float* partial, int m, int64_t n,
-                          int64_t k, uint16_t* y, int64_t ldy, float* yf, int32_t* error,
+                          int64_t k, uint16_t* y, int64_t ldy, int32_t* error,
                           cudaStream_t stream) {
     const int tiles = (int)((n + kRows - 1) / kRows);
     const int splits = choose_splits(n, k, sms);
@@ -634,7 +662,6 @@ static int enqueue_weight(EncodeFn encode, int sms, const uint8_t* w, const uint
     memset(&p, 0, sizeof(p));
     p.y = y;
     p.ldy = ldy;
-    p.yf = yf;
     p.n = n;
     p.k = k;
     p.m = m;
@@ -649,11 +676,11 @@ static int enqueue_weight(EncodeFn encode, int sms, const uint8_t* w, const uint
     p.partial = partial;
     nvfp4_tc_kernel<<<tiles * splits, kThreads, smem_bytes(nx), stream>>>(p, tx, tw, ts);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
-    if (splits > 1) {
-        const int64_t total = (int64_t)m * n;
-        const int threads = 256;
-        nvfp4_tc_reduce<<<(unsigned)((total + threads - 1) / threads), threads, 0, stream>>>(
-            partial, descale, y, ldy, yf, n, m, g, splits);
+    if (splits > 1 && y) {
+        const dim3 grid((unsigned)((n + 4 * kReduceThreads - 1) / (4 * kReduceThreads)),
+                        (unsigned)m);
+        nvfp4_tc_reduce<<<grid, kReduceThreads, 0, stream>>>(partial, descale, y, ldy, n, m, g,
+                                                             splits);
         if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
     }
     return NVFP4_OK;
@@ -675,7 +702,7 @@ int launch(EncodeFn encode, int sms, const uint8_t* w, const uint8_t* s, float g
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
     return enqueue_weight(encode, sms, w, s, g, x16, descale,
                           reinterpret_cast<float*>(base + sc.partial), m, n, k,
-                          static_cast<uint16_t*>(y), ldy, nullptr, static_cast<int32_t*>(ws), stream);
+                          static_cast<uint16_t*>(y), ldy, static_cast<int32_t*>(ws), stream);
 }
 
 int launch_dual(EncodeFn encode, int sms, const uint8_t* wg, const uint8_t* sg, float gg,
@@ -689,22 +716,22 @@ int launch_dual(EncodeFn encode, int sms, const uint8_t* wg, const uint8_t* sg, 
     char* const base = static_cast<char*>(ws) + scratch_off;
     uint16_t* const x16 = reinterpret_cast<uint16_t*>(base + sc.x16);
     float* const descale = reinterpret_cast<float*>(base + sc.descale);
-    float* const partial = reinterpret_cast<float*>(base + sc.partial);
-    float* const gate = reinterpret_cast<float*>(base + sc.gate);
-    float* const up = reinterpret_cast<float*>(base + sc.up);
+    float* const pg = reinterpret_cast<float*>(base + sc.partial);
+    float* const pu = reinterpret_cast<float*>(base + sc.partial_up);
     int32_t* const error = static_cast<int32_t*>(ws);
     nvfp4_tc_prep<<<m, 512, 0, stream>>>(static_cast<const uint16_t*>(x), ldx, k, x16, descale,
                                          pro);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
-    if ((st = enqueue_weight(encode, sms, wg, sg, gg, x16, descale, partial, m, n, k, nullptr, 0,
-                             gate, error, stream)) != NVFP4_OK)
+    // both streams as fp32 partial tiles (y null), then one pass forms o
+    if ((st = enqueue_weight(encode, sms, wg, sg, gg, x16, descale, pg, m, n, k, nullptr, 0,
+                             error, stream)) != NVFP4_OK)
         return st;
-    if ((st = enqueue_weight(encode, sms, wu, su, gu, x16, descale, partial, m, n, k, nullptr, 0,
-                             up, error, stream)) != NVFP4_OK)
+    if ((st = enqueue_weight(encode, sms, wu, su, gu, x16, descale, pu, m, n, k, nullptr, 0,
+                             error, stream)) != NVFP4_OK)
         return st;
-    const int64_t total = (int64_t)m * n;
-    nvfp4_tc_silu_mul<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(
-        gate, up, static_cast<uint16_t*>(y), ldy, n, m, gg, gu);
+    const dim3 grid((unsigned)((n + 4 * kReduceThreads - 1) / (4 * kReduceThreads)), (unsigned)m);
+    nvfp4_tc_dual_finish<<<grid, kReduceThreads, 0, stream>>>(
+        pg, pu, descale, static_cast<uint16_t*>(y), ldy, n, m, gg, gu, choose_splits(n, k, sms));
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
     return NVFP4_OK;
 }
@@ -733,7 +760,7 @@ int launch_multi(EncodeFn encode, int sms, const uint8_t* const* w, const uint8_
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
     for (int o = 0; o < count; ++o)
         if ((st = enqueue_weight(encode, sms, w[o], s[o], g[o], x16, descale, partial, m, n[o], k,
-                                 static_cast<uint16_t*>(y[o]), ldy[o], nullptr,
+                                 static_cast<uint16_t*>(y[o]), ldy[o],
                                  static_cast<int32_t*>(ws), stream)) != NVFP4_OK)
             return st;
     return NVFP4_OK;
