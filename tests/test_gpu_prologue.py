@@ -240,3 +240,65 @@ def test_prologue_beyond_one_register_round():
     y = bits(nv.gemv(W, S, g, dev_x(x), prologue=nv.SigmoidGate(dev_x(t))))
     xo, near = oracle.sigmoid_gate(x, t)
     check_pro_single(y, w, xo, near, "gate, K = 17408")
+
+
+def test_prologue_chain_with_programmatic_launch_and_graphs():
+    # a layer's chain: qkv-like GEMV after a norm (writes h1), an o-like GEMV after the sigmoid
+    # gate, whose output feeds the dual after a norm with h1 as the residual (writes h2); run
+    # plain, with programmatic dependent launch, and as a replayed CUDA graph: all bitwise equal
+    k, m, eps = 1024, 4, 1e-6
+    wq = synth.nvfp4_weight(50, 0, 1536, k)
+    wo = synth.nvfp4_weight(50, 10_000_000, k, k)
+    wg = synth.nvfp4_weight(50, 20_000_000, 2048, k)
+    wu = synth.nvfp4_weight(50, 30_000_000, 2048, k)
+    x, r, gamma1 = norm_inputs(50, m, k)
+    gamma2 = synth.norm_gains(50, 340_000_000, k)
+    a = synth.activations(50, 350_000_000, m, k)
+    t = synth.gate_logits(50, 360_000_000, m, k)
+    Wq, Wo, Wg, Wu = (dev_weight(w) for w in (wq, wo, wg, wu))
+    dx, dr, da, dt = dev_x(x), dev_x(r), dev_x(a), dev_x(t)
+    g1, g2 = dev_vec(gamma1), dev_vec(gamma2)
+    ws = torch.zeros(nv.workspace_bytes_wide(2048, k, m), dtype=torch.uint8, device="cuda")
+    outs = {n_: torch.empty(shape, dtype=torch.bfloat16, device="cuda") for n_, shape in
+            (("q", (m, 1536)), ("o", (m, k)), ("gu", (m, 2048)), ("h1", (m, k)), ("h2", (m, k)))}
+
+    def chain(pdl, stream=None):
+        nv.gemv(*Wq, dx, y=outs["q"], ws=ws, stream=stream, prefetch_weights=pdl,
+                prologue=nv.AddRmsNorm(dr, g1, eps, outs["h1"]))
+        nv.gemv(*Wo, da, y=outs["o"], ws=ws, stream=stream, prefetch_weights=pdl,
+                prologue=nv.SigmoidGate(dt))
+        nv.gemv_dual(*Wg, *Wu, outs["o"], y=outs["gu"], ws=ws, stream=stream,
+                     prefetch_weights=pdl, prologue=nv.AddRmsNorm(outs["h1"], g2, eps, outs["h2"]))
+
+    def snapshot():
+        torch.cuda.synchronize()
+        return {n_: bits(v) for n_, v in outs.items()}
+
+    chain(False)
+    ref = snapshot()
+    for v in outs.values():
+        v.fill_(float("nan"))
+    chain(True)
+    assert all(np.array_equal(ref[n_], got) for n_, got in snapshot().items()), "with PDL"
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        chain(True, s)  # warm-up on the capture stream
+    s.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        chain(True, torch.cuda.current_stream())
+    for v in outs.values():
+        v.fill_(float("nan"))
+    for _ in range(3):
+        graph.replay()
+    assert all(np.array_equal(ref[n_], got) for n_, got in snapshot().items()), "graph replay"
+    del graph
+    # the chain against the oracle: h1, then the gate's GEMV, then the dual on its output
+    h1, xn1, near1 = oracle.add_rmsnorm(x, r, gamma1, eps)
+    assert np.array_equal(ref["h1"], h1)
+    check_pro_single(ref["q"], wq, xn1, near1, "chain q")
+    xo, neargate = oracle.sigmoid_gate(a, t)
+    check_pro_single(ref["o"], wo, xo, neargate, "chain o")
+    h2, xn2, near2 = oracle.add_rmsnorm(ref["o"], h1, gamma2, eps)
+    assert np.array_equal(ref["h2"], h2)
+    check_pro_dual(ref["gu"], wg, wu, xn2, near2, "chain gate_up")
