@@ -227,8 +227,9 @@ typedef struct {
  * x' of a row is computed once and the GEMV's result is that of nvfp4_gemv on x'.  The
  * prologue's arrays are device memory: every row 16-byte aligned (base 16-byte aligned,
  * leading dimension >= K and a multiple of 8), like x.  residual_out may not
- * overlap x, residual, gamma, the gate or any y (rows a launch reads while others write), and
- * residual may not overlap y: NVFP4_ERR_ALIAS.  With NVFP4_FLAG_WIDE_TENSOR the tier's x pass
+ * overlap x, residual, gamma or any y, and residual may not overlap y: NVFP4_ERR_ALIAS (the
+ * prologue may read x and the residual again after writing h, and y is written after it; so
+ * the residual is not updated in place).  With NVFP4_FLAG_WIDE_TENSOR the tier's x pass
  * applies the same prologue, and its rows are invariant over 9..128 as without one.
  * Errors: those of the call without a prologue, and NVFP4_ERR_SHAPE (unknown kind, eps
  * negative or not finite, a leading dimension < K), NVFP4_ERR_NULL (a required array NULL when
