@@ -1163,7 +1163,7 @@ WIDE_ROWS = (16, 32, 64, 128)
 WIDE_DESC = ("sweep layer 0 {qkv 10240x5120, o 5120x6144, gate_up dual 2x17408x5120, down "
              "5120x17408} NVFP4 at M in {16,32,64,128} rows, back to back on one stream, in two "
              "modes: 8-row kernel passes, and the tensor-core tier (NVFP4_FLAG_WIDE_TENSOR) for "
-             "the single-output projections; value: the tier at M = 128")
+             "all four; value: the tier at M = 128")
 
 
 def run_wide(args, world, rank, local):
@@ -1215,7 +1215,68 @@ def run_wide(args, world, rank, local):
                                        ClockSampler(local) if mode == "tensor_tier" else None)
     peak, peak_src = peaks()
     top = per_mode["tensor_tier"][WIDE_ROWS[-1]]
-    return {"metric": METRIC, "value": top["GBps"], "unit": "GB/s", "n_gpus": world,
+    m = WIDE_ROWS[-1]
+
+    # end to end through the public API at M = 128 on the tier: every projection's x in from
+    # pinned host memory, every y back, per step
+    hx = torch.cat([e["x"].reshape(-1) for e in ents]).cpu().pin_memory()
+    dx = torch.empty_like(hx, device=dev)
+    xs, off = [], 0
+    for e in ents:
+        xs.append(dx[off:off + e["x"].numel()].view(e["x"].shape))
+        off += e["x"].numel()
+    hy = [torch.empty_like(e["y"], device="cpu").pin_memory() for e in ents]
+    cur = torch.cuda.current_stream()
+
+    def e2e_step():
+        dx.copy_(hx, non_blocking=True)
+        for e, x in zip(ents, xs):
+            p = e["p"]
+            if p.dual:
+                nv.gemv_dual(e["W"], e["S"], p.w.g, e["Wu"], e["Su"], p.w_up.g, x, y=e["y"],
+                             ws=ws, stream=cur, wide_tensor=True)
+            else:
+                nv.gemv(e["W"], e["S"], p.w.g, x, y=e["y"], ws=ws, stream=cur, wide_tensor=True)
+        for e, h in zip(ents, hy):
+            h.copy_(e["y"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(cur)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    t1.record(cur)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(t0.elapsed_time(t1), world) / args.e2e_steps
+    step_b = top["GBps"] * 1e9 * top["ms_per_step"] * 1e-3 / world
+    e2e = {"value": round(world * step_b / (ms_e2e * 1e-3) / 1e9, 1), "unit": "GB/s",
+           "h2d_bytes_per_step": hx.numel() * 2,
+           "d2h_bytes_per_step": sum(e["y"].numel() * 2 for e in ents), "steps": args.e2e_steps,
+           "api": "nvfp4_weight_only_03_b200.gemv / gemv_dual with wide_tensor=True, M = 128"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        threads = os.cpu_count() or 1
+        qkv = projs[0]
+        xb = synth.activations(wl.seed + 100, 0, m, qkv.k)
+        t_end = time.perf_counter() + args.cpu_seconds
+        b, n_calls, t_start = 0, 0, time.perf_counter()
+        while time.perf_counter() < t_end:
+            oracle.gemv(qkv.w.packed, qkv.w.scales, qkv.w.g, xb, rows=np.arange(64),
+                        threads=threads)
+            b += 64 * (qkv.k // 2 + qkv.k // 16) + m * qkv.k * 2 + m * 64 * 2
+            n_calls += 1
+        dt = time.perf_counter() - t_start
+        cpu = {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n_calls} calls of 64 qkv output rows at M = {m} ({dt:.1f} s)"}
+
+    line = {"metric": METRIC, "value": top["GBps"], "unit": "GB/s", "n_gpus": world,
             "steps": top["steps"], "warmup": args.warmup, "ms_per_step": top["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "nvfp4(e2m1+e4m3) x bf16 -> fp32 accumulate, bf16 out",
@@ -1230,7 +1291,10 @@ def run_wide(args, world, rank, local):
             "per_rows": per_mode,
             "gpu_launches": (top["kernels_per_step"] * top["steps"]
                              if top.get("kernels_per_step") is not None else None),
-            "clocks": top.get("clocks")}
+            "clocks": top.get("clocks"), "e2e": e2e}
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    return line
 
 
 def peaks_bf16():
