@@ -302,3 +302,25 @@ def test_prologue_chain_with_programmatic_launch_and_graphs():
     h2, xn2, near2 = oracle.add_rmsnorm(ref["o"], h1, gamma2, eps)
     assert np.array_equal(ref["h2"], h2)
     check_pro_dual(ref["gu"], wg, wu, xn2, near2, "chain gate_up")
+
+
+def test_prologue_with_multi_on_the_tier():
+    # q, k, v sharing the normed x at M = 24 on the tier: each output bitwise its own
+    # single-output call with the same prologue, and within tolerance of the oracle
+    k, m, eps = 5120, 24, 1e-6
+    ws_ = [synth.nvfp4_weight(51, off, n, k) for off, n in
+           ((0, 2048), (20_000_000, 1024), (30_000_000, 1024))]
+    x, r, gamma = norm_inputs(51, m, k)
+    devs = [dev_weight(w) for w in ws_]
+    h_out = torch.empty((m, k), dtype=torch.bfloat16, device="cuda")
+    ys = [bits(y) for y in nv.gemv_multi(devs, dev_x(x), wide_tensor=True, prologue=nv.AddRmsNorm(
+        dev_x(r), dev_vec(gamma), eps, h_out))]
+    h_ref, xn, near = oracle.add_rmsnorm(x, r, gamma, eps)
+    assert np.array_equal(bits(h_out), h_ref)
+    for o, (w, d) in enumerate(zip(ws_, devs)):
+        single = bits(nv.gemv(*d, dev_x(x), wide_tensor=True,
+                              prologue=nv.AddRmsNorm(dev_x(r), dev_vec(gamma), eps)))
+        assert np.array_equal(ys[o], single), f"output {o}"
+        rows = sample_rows(w.n, 100) if w.n > 2048 else None
+        check_pro_single(ys[o] if rows is None else ys[o][:, rows], w, xn, near,
+                         f"multi tier output {o}", rows)
