@@ -18,6 +18,9 @@ Parity status of each function (what pins it is listed in the tests named here):
                              50-digit decimal brute force (tests/test_oracle_prologue.py)
   sigmoid_gate ............. pinned: sigmoid(0) = 1/2, saturation, the symmetry
                              sigmoid(t) + sigmoid(-t) = 1, decimal brute force (same file)
+  gated_rmsnorm ............ pinned: closed forms of a constant group and of the gate, group
+                             independence, scale invariance per group, decimal brute force
+                             (same file)
 """
 from __future__ import annotations
 
@@ -68,6 +71,9 @@ def _load():
         lib.oracle_add_rmsnorm.restype = c_int
         lib.oracle_sigmoid_gate.argtypes = [vp, i64, vp, i64, c_int, i64, vp, vp]
         lib.oracle_sigmoid_gate.restype = c_int
+        lib.oracle_gated_rmsnorm.argtypes = [vp, i64, vp, i64, vp, c_int, ctypes.c_float, c_int,
+                                             i64, vp, vp]
+        lib.oracle_gated_rmsnorm.restype = c_int
         _lib = lib
     return _lib
 
@@ -194,6 +200,25 @@ def sigmoid_gate(a, gate):
     rc = _load().oracle_sigmoid_gate(pa, k, pg, k, m, k, xo.ctypes.data, near.ctypes.data)
     if rc:
         raise ValueError("oracle_sigmoid_gate rejected its arguments")
+    return xo, near
+
+
+def gated_rmsnorm(x, z, gamma, group: int, eps: float):
+    """Gated RMS norm per group of channels (x: fp32 [m][k]; z: bf16 bits [m][k]; gamma: bf16
+    bits [group]).  Returns (xo, near): xo = bf16(x gamma silu(z) / sqrt(mean_group(x^2) + eps))
+    as bf16 bits [m][k], and the near-midpoint mask."""
+    x, px = _c(np.atleast_2d(x), np.float32)
+    z, pz = _c(np.atleast_2d(z), np.uint16)
+    gamma, pg = _c(gamma, np.uint16)
+    m, k = x.shape
+    if z.shape != (m, k) or gamma.shape != (group,):
+        raise ValueError("x and z must be [m][k], gamma [group]")
+    xo = np.zeros((m, k), np.uint16)
+    near = np.zeros((m, k), np.uint8)
+    rc = _load().oracle_gated_rmsnorm(px, k, pz, k, pg, group, eps, m, k, xo.ctypes.data,
+                                      near.ctypes.data)
+    if rc:
+        raise ValueError("oracle_gated_rmsnorm rejected its arguments")
     return xo, near
 
 

@@ -28,6 +28,10 @@
  * the sigmoid output gate of gated attention):
  *   add + RMS norm:  h = bf16(x + r);  xn = bf16(h * gamma / sqrt(mean_k(h^2) + eps))
  *   sigmoid gate:    xo = bf16(a * sigmoid(gate)),  sigmoid(t) = 1 / (1 + exp(-t))
+ *   gated RMS norm ("gated_rms_norm_f32_input", the GatedDeltaNet's output norm before its
+ *   output projection): x in fp32, normalised per group of G channels (one head),
+ *                    xo = bf16(x * gamma[k mod G] * silu(z) / sqrt(mean_group(x^2) + eps)),
+ *                    silu(t) = t / (1 + exp(-t))
  * in fp64 with one rounding to bf16 at the end of each line.
  *
  * Formats, written from their definitions (the pages name the format, not its bits):
@@ -221,6 +225,37 @@ int oracle_sigmoid_gate(const uint16_t* a, int64_t lda, const uint16_t* gate, in
             uint16_t b = oracle_bf16_rne(v);
             xo[i * k + j] = b;
             if (near) near[i * k + j] = near_midpoint(v, b);
+        }
+    return 0;
+}
+
+/* Gated RMS norm over groups of `group` channels: for row i and group q (channels q*group ..),
+ *   ms = (1/group) sum x^2 over the group (fp64, increasing k)
+ *   xo[i][k] = bf16_rne(x[i][k] * gamma[k % group] * silu(z[i][k]) / sqrt(ms + eps))
+ * x is fp32 [m][ldx], z bf16 [m][ldz], gamma bf16 [group]; xo is [m][k]; near as above. */
+int oracle_gated_rmsnorm(const float* x, int64_t ldx, const uint16_t* z, int64_t ldz,
+                         const uint16_t* gamma, int group, float eps, int m, int64_t k,
+                         uint16_t* xo, uint8_t* near) {
+    if (m < 0 || k <= 0 || group <= 0 || (k % group) || ldx < k || ldz < k || !x || !z ||
+        !gamma || !xo)
+        return -1;
+    if (!(eps >= 0.0f) || isinf(eps)) return -1;
+    for (int i = 0; i < m; ++i)
+        for (int64_t q0 = 0; q0 < k; q0 += group) {
+            double ss = 0.0;
+            for (int j = 0; j < group; ++j) {
+                double v = (double)x[i * ldx + q0 + j];
+                ss += v * v;
+            }
+            double inv = 1.0 / sqrt(ss / (double)group + (double)eps);
+            for (int j = 0; j < group; ++j) {
+                double t = oracle_bf16_value(z[i * ldz + q0 + j]);
+                double silu = t / (1.0 + exp(-t));
+                double v = (double)x[i * ldx + q0 + j] * oracle_bf16_value(gamma[j]) * silu * inv;
+                uint16_t b = oracle_bf16_rne(v);
+                xo[i * k + q0 + j] = b;
+                if (near) near[i * k + q0 + j] = near_midpoint(v, b);
+            }
         }
     return 0;
 }

@@ -206,3 +206,73 @@ def test_rounding_slack_is_the_neighbour_gap_where_near():
     near = np.array([[1, 0, 1, 0]], np.uint8)
     s = val(oracle.rounding_slack(xq, near))
     assert list(s[0]) == [2 ** -7, 0.0, 2 ** -6, 0.0]
+
+
+# ---- gated RMS norm (per group of channels, fp32 input, SiLU gate)
+
+def test_gated_rmsnorm_closed_forms():
+    # a constant group normalises to +-1; gate 100 passes through silu(100) = 100 (to fp64);
+    # gamma 1/4: x' = +-25 exactly, group by group
+    g = 128
+    x = np.array([[1.5] * g + [-0.25] * g + [3e-3] * g], np.float32)
+    z = bf(np.full((1, 3 * g), 100.0))
+    gamma = bf(np.full(g, 0.25))
+    xo, _ = oracle.gated_rmsnorm(x, z, gamma, g, 0.0)
+    assert list(np.unique(val(xo[0, :g]))) == [25.0]
+    assert list(np.unique(val(xo[0, g:2 * g]))) == [-25.0]
+    assert list(np.unique(val(xo[0, 2 * g:]))) == [25.0]
+    # gate 0: silu(0) = 0 gives signed zeros
+    xo, _ = oracle.gated_rmsnorm(x, np.zeros_like(z), gamma, g, 0.0)
+    assert not val(xo).any()
+    # eps inside the square root: constant c with eps = 3 c^2 halves the result
+    c = 2.0 ** -6
+    xo, _ = oracle.gated_rmsnorm(np.full((1, g), c, np.float32), bf(np.full((1, g), 100.0)),
+                                 gamma, g, 3 * c * c)
+    assert list(np.unique(val(xo))) == [12.5]
+
+
+def test_gated_rmsnorm_groups_are_independent_and_scale_free():
+    rng = np.random.default_rng(7)
+    g, m = 128, 2
+    x = rng.normal(0, 1, (m, 4 * g)).astype(np.float32)
+    z = bf(rng.normal(0, 2, (m, 4 * g)))
+    gamma = bf(rng.uniform(0.5, 1.5, g))
+    xo, _ = oracle.gated_rmsnorm(x, z, gamma, g, 0.0)
+    # changing group 2 leaves the other groups unchanged
+    x2 = x.copy()
+    x2[:, 2 * g:3 * g] *= 7.0
+    xo2, _ = oracle.gated_rmsnorm(x2, z, gamma, g, 0.0)
+    keep = np.r_[0:2 * g, 3 * g:4 * g]
+    assert np.array_equal(xo2[:, keep], xo[:, keep])
+    # scaling a group by a power of two leaves its x' unchanged (eps = 0)
+    x3 = x.copy()
+    x3[:, g:2 * g] *= np.float32(2.0 ** 20)
+    xo3, _ = oracle.gated_rmsnorm(x3, z, gamma, g, 0.0)
+    assert np.array_equal(xo3, xo)
+    # one group of a wider row equals the same values as a row of their own
+    xo4, _ = oracle.gated_rmsnorm(x[:, g:2 * g], z[:, g:2 * g], gamma, g, 0.0)
+    assert np.array_equal(xo4, xo[:, g:2 * g])
+
+
+@decimal_digits(50)
+def test_gated_rmsnorm_decimal_brute_force():
+    rng = np.random.default_rng(8)
+    g, m = 32, 2
+    x = rng.normal(0, 1, (m, 2 * g)).astype(np.float32)
+    z = bf(rng.normal(0, 2, (m, 2 * g)))
+    gamma = bf(rng.uniform(0.5, 1.5, g))
+    eps = float(np.float32(1e-5))
+    xo, near = oracle.gated_rmsnorm(x, z, gamma, g, eps)
+    for i in range(m):
+        for q in range(2):
+            xs = [Decimal(float(v)) for v in x[i, q * g:(q + 1) * g]]
+            inv = 1 / (sum(v * v for v in xs) / g + Decimal(eps)).sqrt()
+            for j in range(g):
+                t = Decimal(float(val(z[i, q * g + j])))
+                silu = t / (1 + (-t).exp())
+                want = dec_to_bf16(xs[j] * Decimal(float(val(gamma[j]))) * silu * inv)
+                got = int(xo[i, q * g + j])
+                if near[i, q * g + j]:
+                    assert abs(oracle.bf16_ordinal(got) - oracle.bf16_ordinal(want)) <= 1
+                else:
+                    assert got == want, (i, q, j)
