@@ -66,12 +66,12 @@ def parse():
 # launch, for layer 0 of the sweep at M = 1 and M = 8 (profiles/nvfp4_gemv_sweep_dram_traffic.md).
 # They describe the kernel code with this SHA-256 only (kernel_code_sha256: comments and blank
 # lines do not count); for any other code the bench reports traffic as null.
-TRAFFIC_SOURCE_SHA256 = "f93c361d24e4656960e8b9966fe0f77a3dcce9c44015611b0fc567fe4d7ca6f8"
+TRAFFIC_SOURCE_SHA256 = "d1b5f55b5d018df462518828592786b8db2e8e99ec64e00852a2de8f26c49be8"
 TRAFFIC_BYTES = {
-    ("L0.qkv", 1): 30119168, ("L0.o", 1): 18323968, ("L0.gate_up", 1): 107118848,
-    ("L0.down", 1): 50808320,
-    ("L0.qkv", 8): 29617408, ("L0.o", 8): 17837312, ("L0.gate_up", 8): 105671168,
-    ("L0.down", 8): 50468608,
+    ("L0.qkv", 1): 30119168, ("L0.o", 1): 18324480, ("L0.gate_up", 1): 106684416,
+    ("L0.down", 1): 50807296,
+    ("L0.qkv", 8): 29617152, ("L0.o", 8): 17837312, ("L0.gate_up", 8): 105905152,
+    ("L0.down", 8): 50465024,
 }
 KERNEL_SOURCE = os.path.join(ROOT, "nvfp4_weight_only_03_b200", "csrc", "nvfp4_gemv.cu")
 

@@ -196,6 +196,14 @@ int nvfp4_gemv_multi(const nvfp4_output_t* outputs, int count, const void* x, in
  *                                 inv(m)   = 1 / sqrt(sum_k h[m][k]^2 / K + eps)
  *                                 and h is written to residual_out when that is not NULL.
  *   NVFP4_PROLOGUE_SIGMOID_GATE:  x'[m][k] = bf16_rn(x[m][k] / (1 + e^-gate[m][k]))
+ *   NVFP4_PROLOGUE_GATED_RMSNORM: x is fp32 [M][ldx] for this kind (the GatedDeltaNet's
+ *                                 output, "gated_rms_norm_f32_input" on the same page), and
+ *                                 every group of G = `group` channels is normalised alone:
+ *                                 x'[m][k] = bf16_rn(x[m][k] * inv(m, g) * gamma[k mod G]
+ *                                                    * silu(gate[m][k])),
+ *                                 inv(m, g) = 1 / sqrt(sum_{k in g} x[m][k]^2 / G + eps),
+ *                                 silu(t) = t / (1 + e^-t).  G % 128 == 0, G <= 512,
+ *                                 K % G == 0; NVFP4_FLAG_WIDE_TENSOR is ignored (8-row passes).
  *
  * in fp32 (h exactly rounded; the sum of squares in a fixed order).  gamma multiplies as given:
  * a checkpoint that stores (gamma - 1) passes 1 + its weights.  Row invariance over M = 1..128
@@ -204,19 +212,21 @@ int nvfp4_gemv_multi(const nvfp4_output_t* outputs, int count, const void* x, in
 typedef enum {
     NVFP4_PROLOGUE_NONE = 0,
     NVFP4_PROLOGUE_ADD_RMSNORM = 1,
-    NVFP4_PROLOGUE_SIGMOID_GATE = 2
+    NVFP4_PROLOGUE_SIGMOID_GATE = 2,
+    NVFP4_PROLOGUE_GATED_RMSNORM = 3
 } nvfp4_prologue_kind;
 
 typedef struct {
     int32_t kind;            /* nvfp4_prologue_kind */
-    float eps;               /* ADD_RMSNORM: finite, >= 0 */
+    float eps;               /* ADD_RMSNORM, GATED_RMSNORM: finite, >= 0 */
     const void* residual;    /* ADD_RMSNORM: bf16 [M][ld_residual] */
     int64_t ld_residual;
-    const void* gamma;       /* ADD_RMSNORM: bf16 [K] */
+    const void* gamma;       /* ADD_RMSNORM: bf16 [K]; GATED_RMSNORM: bf16 [G] */
     void* residual_out;      /* ADD_RMSNORM: bf16 [M][ld_residual_out] receives h, or NULL */
     int64_t ld_residual_out;
-    const void* gate;        /* SIGMOID_GATE: bf16 [M][ld_gate] */
+    const void* gate;        /* SIGMOID_GATE, GATED_RMSNORM: bf16 [M][ld_gate] */
     int64_t ld_gate;
+    int32_t group;           /* GATED_RMSNORM: channels per group, G (gamma is bf16 [G]) */
 } nvfp4_prologue_t;
 
 /* nvfp4_gemv_ex, nvfp4_gemv_dual_ex and nvfp4_gemv_multi with an input prologue.  `prologue`

@@ -55,10 +55,11 @@ class Prologue(ctypes.Structure):
                 ("residual", ctypes.c_void_p), ("ld_residual", ctypes.c_int64),
                 ("gamma", ctypes.c_void_p),
                 ("residual_out", ctypes.c_void_p), ("ld_residual_out", ctypes.c_int64),
-                ("gate", ctypes.c_void_p), ("ld_gate", ctypes.c_int64)]
+                ("gate", ctypes.c_void_p), ("ld_gate", ctypes.c_int64),
+                ("group", ctypes.c_int32)]
 
 
-PROLOGUE_NONE, PROLOGUE_ADD_RMSNORM, PROLOGUE_SIGMOID_GATE = 0, 1, 2
+PROLOGUE_NONE, PROLOGUE_ADD_RMSNORM, PROLOGUE_SIGMOID_GATE, PROLOGUE_GATED_RMSNORM = 0, 1, 2, 3
 
 
 def _rows_arg(t: torch.Tensor, m: int, k: int, name: str):
@@ -90,6 +91,25 @@ class AddRmsNorm:
             h, ldh = _rows_arg(self.residual_out, m, k, "residual_out")
             p.residual_out, p.ld_residual_out = h.data_ptr(), ldh
         return p
+
+
+class GatedRmsNorm:
+    """Prologue for an fp32 x (pass x as float32): every group of `group` channels is normalised
+    alone, x' = bf16(x / sqrt(mean_group(x^2) + eps) * gamma[k % group] * silu(gate)).
+    group % 128 == 0, group <= 512; gamma is bfloat16 [group], gate bfloat16 [M][K]."""
+
+    x_dtype = torch.float32
+
+    def __init__(self, gate: torch.Tensor, gamma: torch.Tensor, group: int, eps: float = 1e-6):
+        self.gate, self.gamma, self.group, self.eps = gate, gamma, group, eps
+
+    def struct(self, m: int, k: int) -> Prologue:
+        t, ldt = _rows_arg(self.gate, m, k, "gate")
+        if self.gamma.dtype != torch.bfloat16 or self.gamma.shape != (self.group,) or \
+                not self.gamma.is_contiguous():
+            raise ValueError(f"gamma must be contiguous bfloat16 [{self.group}]")
+        return Prologue(kind=PROLOGUE_GATED_RMSNORM, eps=float(self.eps), gate=t.data_ptr(),
+                        ld_gate=ldt, gamma=self.gamma.data_ptr(), group=int(self.group))
 
 
 class SigmoidGate:
@@ -219,9 +239,9 @@ def _weight_args(w: torch.Tensor, s: torch.Tensor):
     return n, k
 
 
-def _x_args(x: torch.Tensor, k: int):
-    if x.dtype != torch.bfloat16:
-        raise TypeError("x must be bfloat16")
+def _x_args(x: torch.Tensor, k: int, dtype=torch.bfloat16):
+    if x.dtype != dtype:
+        raise TypeError(f"x must be {dtype}")
     if x.dim() == 1:
         x = x.unsqueeze(0)
     if x.dim() != 2 or x.shape[1] != k or x.stride(1) != 1:
@@ -266,7 +286,7 @@ def gemv(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor, y: torch.T
     prologue: AddRmsNorm or SigmoidGate, applied to x inside the call (its x' lives in the
     workspace, so a caller's ws must hold workspace_bytes_wide(n, k, m))."""
     n, k = _weight_args(w, s)
-    x, m, ldx = _x_args(x, k)
+    x, m, ldx = _x_args(x, k, getattr(prologue, "x_dtype", torch.bfloat16))
     pro = None if prologue is None else prologue.struct(m, k)
     y, ldy = _out(y, m, n, x)
     if ws is None:
@@ -308,7 +328,7 @@ def gemv_dual(wg: torch.Tensor, sg: torch.Tensor, gg: float, wu: torch.Tensor, s
     n, k = _weight_args(wg, sg)
     if _weight_args(wu, su) != (n, k):
         raise ValueError("gate and up weights must have the same shape")
-    x, m, ldx = _x_args(x, k)
+    x, m, ldx = _x_args(x, k, getattr(prologue, "x_dtype", torch.bfloat16))
     pro = None if prologue is None else prologue.struct(m, k)
     y, ldy = _out(y, m, n, x)
     if ws is None:
@@ -340,7 +360,7 @@ def gemv_multi(weights, x: torch.Tensor, ys=None, ws: torch.Tensor = None, strea
     k = shapes[0][1]
     if any(kk != k for _, kk in shapes):
         raise ValueError("all weights must have the same K")
-    x, m, ldx = _x_args(x, k)
+    x, m, ldx = _x_args(x, k, getattr(prologue, "x_dtype", torch.bfloat16))
     pro = None if prologue is None else prologue.struct(m, k)
     ys = [None] * len(weights) if ys is None else list(ys)
     if len(ys) != len(weights):

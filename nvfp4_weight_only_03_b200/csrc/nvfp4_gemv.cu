@@ -530,8 +530,9 @@ __global__ void __launch_bounds__(Cfg<DUAL>::kThreads, 1)
         if (r < p.m)
             for (int c = part * 32 + lane; c < per_row; c += wpr * 32) {
                 const uint4 v = xsm[r * xrow + c];
-                a = max(a, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                                    __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
+                // per-halfword maximum (two bf16 magnitudes per word), folded below
+                a = __vmaxu2(a, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                         __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
             }
         a = max(a & 0xFFFFu, a >> 16);
 #pragma unroll
@@ -744,13 +745,48 @@ constexpr int kProThreads = 512;
 constexpr int kProKeep = 4;  // chunks a thread keeps in registers between the two passes
 
 __global__ void __launch_bounds__(kProThreads)
-    nvfp4_prologue_kernel(const nvfp4_pro::Prologue pro, const uint16_t* __restrict__ x,
+    nvfp4_prologue_kernel(const nvfp4_pro::Prologue pro, const void* __restrict__ xv,
                           int64_t ldx, int64_t k, uint16_t* __restrict__ xo) {
     pdl_launch_dependents();
     pdl_wait();  // x and the prologue's arrays may come from the preceding kernel
     __shared__ float s_red[kProThreads / 32];
     __shared__ float s_inv;
     const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (pro.kind == NVFP4_PROLOGUE_GATED_RMSNORM) {
+        // x fp32: a warp per group of G channels (groups w, w + 16, ...); lane l holds elements
+        // 4 (l + 32 i) .. +3 for i < G / 128, sums their squares in element order, then a fixed
+        // xor tree over the warp
+        const float* xr = static_cast<const float*>(xv) + m * ldx;
+        const uint16_t* zr = pro.in + m * pro.ld_in;
+        uint16_t* outr = xo + m * k;
+        const int g = pro.group, q = g / 128;
+        for (int64_t g0 = (int64_t)warp * g; g0 < k; g0 += (int64_t)(kProThreads / 32) * g) {
+            float4 v[4];
+            float ss = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (i < q) {
+                    v[i] = *reinterpret_cast<const float4*>(xr + g0 + 4 * (lane + 32 * i));
+                    ss = fmaf(v[i].x, v[i].x, ss);
+                    ss = fmaf(v[i].y, v[i].y, ss);
+                    ss = fmaf(v[i].z, v[i].z, ss);
+                    ss = fmaf(v[i].w, v[i].w, ss);
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+            const float inv = nvfp4_pro::rms_inverse(ss, g, pro.eps);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (i < q) {
+                    const int e = 4 * (lane + 32 * i);
+                    *reinterpret_cast<uint2*>(outr + g0 + e) = nvfp4_pro::gated_4(
+                        v[i], *reinterpret_cast<const uint2*>(zr + g0 + e),
+                        *reinterpret_cast<const uint2*>(pro.gamma + e), inv);
+                }
+        }
+        return;
+    }
+    const uint16_t* const x = static_cast<const uint16_t*>(xv);
     const int64_t nch = k >> 3;
     const uint4* xr = reinterpret_cast<const uint4*>(x + m * ldx);
     const uint4* ar = reinterpret_cast<const uint4*>(pro.in + m * pro.ld_in);
@@ -923,6 +959,24 @@ int check_pro(const nvfp4_prologue_t* pp, const void* x, int64_t ldx, int m, int
               const Range* ys, int ny, nvfp4_pro::Prologue* out) {
     memset(out, 0, sizeof(*out));
     if (!pp || pp->kind == NVFP4_PROLOGUE_NONE) return NVFP4_OK;
+    if (pp->kind == NVFP4_PROLOGUE_GATED_RMSNORM) {
+        // x is fp32 here: check_common's 16-byte rows and ldx % 8 hold for it too
+        const int g = pp->group;
+        if (!(pp->eps >= 0.0f && pp->eps <= 3.402823466e38f)) return NVFP4_ERR_SHAPE;
+        if (g < 128 || g > 512 || (g % 128) != 0) return NVFP4_ERR_SHAPE;
+        out->kind = pp->kind;
+        out->eps = pp->eps;
+        out->group = g;
+        if (m <= 0 || k <= 0) return NVFP4_OK;
+        if ((k % g) != 0 || pp->ld_gate < k) return NVFP4_ERR_SHAPE;
+        if (!pp->gate || !pp->gamma) return NVFP4_ERR_NULL;
+        if ((pp->ld_gate % 8) != 0 || misaligned(pp->gate, 16) || misaligned(pp->gamma, 16))
+            return NVFP4_ERR_ALIGN;
+        out->in = static_cast<const uint16_t*>(pp->gate);
+        out->ld_in = pp->ld_gate;
+        out->gamma = static_cast<const uint16_t*>(pp->gamma);
+        return NVFP4_OK;
+    }
     const bool norm = pp->kind == NVFP4_PROLOGUE_ADD_RMSNORM;
     if (!norm && pp->kind != NVFP4_PROLOGUE_SIGMOID_GATE) return NVFP4_ERR_SHAPE;
     if (norm && !(pp->eps >= 0.0f && pp->eps <= 3.402823466e38f)) return NVFP4_ERR_SHAPE;
@@ -1201,8 +1255,7 @@ int prologue_pass(const nvfp4_pro::Prologue& pro, const void** x, int64_t* ldx, 
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    if (cudaLaunchKernelEx(&cfg, nvfp4_prologue_kernel, pro, static_cast<const uint16_t*>(*x),
-                           *ldx, k, xo) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, nvfp4_prologue_kernel, pro, *x, *ldx, k, xo) != cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_LAUNCH;
     }
@@ -1274,7 +1327,7 @@ int nvfp4_gemv_pro(const nvfp4_prologue_t* prologue, const uint8_t* w, const uin
     if (noop) return NVFP4_OK;
     if (k > 0 && (st = check_weight(w, s)) != NVFP4_OK) return st;
     if ((flags & NVFP4_FLAG_WIDE_TENSOR) && m > NVFP4_PASS_ROWS && k > 0 &&
-        nvfp4_tc::usable(s, k)) {
+        pro.kind != NVFP4_PROLOGUE_GATED_RMSNORM && nvfp4_tc::usable(s, k)) {
         int dev = 0;
         DeviceInfo* di = nullptr;
         if ((st = device_info(&dev, &di)) != NVFP4_OK) return st;
@@ -1361,7 +1414,8 @@ int nvfp4_gemv_dual_pro(const nvfp4_prologue_t* prologue, const uint8_t* w_gate,
         if ((st = check_weight(w_up, s_up)) != NVFP4_OK) return st;
     }
     if ((flags & NVFP4_FLAG_WIDE_TENSOR) && m > NVFP4_PASS_ROWS && k > 0 &&
-        nvfp4_tc::usable(s_gate, k) && nvfp4_tc::usable(s_up, k)) {
+        pro.kind != NVFP4_PROLOGUE_GATED_RMSNORM && nvfp4_tc::usable(s_gate, k) &&
+        nvfp4_tc::usable(s_up, k)) {
         int dev = 0;
         DeviceInfo* di = nullptr;
         if ((st = device_info(&dev, &di)) != NVFP4_OK) return st;
@@ -1432,7 +1486,8 @@ int nvfp4_gemv_multi_pro(const nvfp4_prologue_t* prologue, const nvfp4_output_t*
     DeviceInfo* di = nullptr;
     st = device_info(&dev, &di);
     if (st != NVFP4_OK) return st;
-    if ((flags & NVFP4_FLAG_WIDE_TENSOR) && m > NVFP4_PASS_ROWS && k > 0) {
+    if ((flags & NVFP4_FLAG_WIDE_TENSOR) && m > NVFP4_PASS_ROWS && k > 0 &&
+        pro.kind != NVFP4_PROLOGUE_GATED_RMSNORM) {
         bool all = true;
         for (int o = 0; o < used; ++o) all = all && nvfp4_tc::usable(sp[o].s[0], k);
         if (all) {

@@ -490,8 +490,9 @@ __global__ void __launch_bounds__(512) nvfp4_tc_prep(const uint16_t* __restrict_
     for (int64_t i = threadIdx.x; i < k8; i += blockDim.x) {
         uint4 v = row[i];
         if (pro.kind != NVFP4_PROLOGUE_NONE) v = nvfp4_pro::apply_8(pro, v, m, 8 * i, inv);
-        a = max(a, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                            __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
+        // per-halfword maximum (two bf16 magnitudes per word), folded below
+        a = __vmaxu2(a, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                 __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
     }
     a = max(a & 0xFFFFu, a >> 16);
 #pragma unroll

@@ -8,6 +8,8 @@
 //   NVFP4_PROLOGUE_ADD_RMSNORM:  h = bf16(x + r);  x' = bf16((h * inv) * gamma),
 //                                inv = 1 / sqrt(sum_k h^2 / K + eps)
 //   NVFP4_PROLOGUE_SIGMOID_GATE: x' = bf16(x / (1 + e^-gate))
+//   NVFP4_PROLOGUE_GATED_RMSNORM: x fp32; x' = bf16(((x * inv_g) * gamma[k mod G]) * silu(z)),
+//                                inv_g = 1 / sqrt(sum_{group} x^2 / G + eps), silu(t) = t / (1 + e^-t)
 //
 // in fp32.  x + r of two bf16 values rounded once to bf16 equals the exactly rounded sum (fp32
 // carries more than twice bf16's precision plus two bits).  Each caller sums a row's squares in
@@ -30,6 +32,7 @@ struct Prologue {
     const uint16_t* gamma; // ADD_RMSNORM: bf16 [K]
     uint16_t* hout;        // ADD_RMSNORM: h = bf16(x + r), bf16 [M][ldh], or null
     int64_t ldh;
+    int group;             // GATED_RMSNORM: channels per group
 };
 
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
@@ -86,6 +89,15 @@ __device__ __forceinline__ uint4 gate_8(uint4 x, uint4 t) {
                       bf2_rn(gated(bf_lo(x.y), bf_lo(t.y)), gated(bf_hi(x.y), bf_hi(t.y))),
                       bf2_rn(gated(bf_lo(x.z), bf_lo(t.z)), gated(bf_hi(x.z), bf_hi(t.z))),
                       bf2_rn(gated(bf_lo(x.w), bf_lo(t.w)), gated(bf_hi(x.w), bf_hi(t.w))));
+}
+
+// x' = bf16(((x * inv) * gamma) * silu(z)) for 4 fp32 values of x, 4 bf16 of z and gamma
+__device__ __forceinline__ uint2 gated_4(float4 x, uint2 z, uint2 g, float inv) {
+    const float z0 = bf_lo(z.x), z1 = bf_hi(z.x), z2 = bf_lo(z.y), z3 = bf_hi(z.y);
+    return make_uint2(bf2_rn(x.x * inv * bf_lo(g.x) * gated(z0, z0),
+                             x.y * inv * bf_hi(g.x) * gated(z1, z1)),
+                      bf2_rn(x.z * inv * bf_lo(g.y) * gated(z2, z2),
+                             x.w * inv * bf_hi(g.y) * gated(z3, z3)));
 }
 
 // The transformed 8 values at (row m, k .. k+7) given x's raw values there.

@@ -279,3 +279,32 @@ def test_prologue_binding_argument_checks():
         nv.gemv(w, s, 1.0, x, prologue=nv.AddRmsNorm(r[:1], torch.ones(64, dtype=torch.bfloat16)))
     with pytest.raises(TypeError):   # gate not bf16
         nv.gemv(w, s, 1.0, x, prologue=nv.SigmoidGate(torch.zeros((2, 64))))
+
+
+def gated(group=128, eps=1e-6, gate=PT, ld_gate=256, gamma=PG):
+    return nv.Prologue(kind=nv.PROLOGUE_GATED_RMSNORM, eps=eps, gate=gate, ld_gate=ld_gate,
+                       gamma=gamma, group=group)
+
+
+@pytest.mark.parametrize("kw,k,status", [
+    (dict(group=64), 256, -2), (dict(group=192), 384, -2), (dict(group=640), 1280, -2),
+    (dict(group=256), 384, -2),              # K % G != 0
+    (dict(eps=-1.0), 256, -2), (dict(eps=float("nan")), 256, -2),
+    (dict(gate=None), 256, -1), (dict(gamma=None), 256, -1),
+    (dict(ld_gate=128), 256, -2), (dict(ld_gate=260), 256, -4),
+    (dict(gate=PT + 8), 256, -4), (dict(gamma=PG + 8), 256, -4),
+])
+def test_gated_rmsnorm_host_checks(L, kw, k, status):
+    p = gated(**kw)
+    if "ld_gate" not in kw:
+        p.ld_gate = k
+    assert L.nvfp4_gemv_pro(ctypes.byref(p), PW, PW, 1.0, PX, k, PY, 64, 2, 64, k, PWS, 1 << 30,
+                            0, None) == status
+
+
+def test_gated_rmsnorm_valid_call_reaches_the_device(L):
+    p = gated()
+    expect = 0 if cuda_ok() else -5
+    if not cuda_ok():
+        assert L.nvfp4_gemv_pro(ctypes.byref(p), PW, PW, 1.0, PX, 256, PY, 64, 2, 64, 256, PWS,
+                                1 << 30, 0, None) == expect

@@ -348,3 +348,43 @@ def test_scale_copy_paths(ws, k, offset):
     check_single(y, ref, a, f"k={k} offset={offset}")
     y0 = bits(nv.gemv(W, torch.from_numpy(w.scales).cuda(), w.g, dev_x(x), ws=ws))
     assert np.array_equal(y, y0)
+
+
+def amax_trap_rows(m, k, k0=1000):
+    """x rows whose largest magnitude sits in the low half of a bf16 pair while other words of
+    the same lane have a larger high half: 1.0 at even k, 3.0 at odd k, and in the 8-element
+    chunk holding k0 (even) 2.0 at odd k and 1000 at k0.  A per-row maximum that compared
+    packed pairs as whole words would miss the 1000 and overflow f16."""
+    v = np.where(np.arange(k) % 2 == 0, 1.0, 3.0)
+    c0 = k0 - k0 % 8
+    v[c0 + 1:c0 + 8:2] = 2.0
+    v[k0] = 1000.0
+    return oracle.bf16_rne(np.tile(v, (m, 1)))
+
+
+@pytest.mark.parametrize("m", [1, 5, 8])
+def test_row_maximum_in_a_low_half_word(m):
+    n, k = 1000, 5120
+    w = synth.nvfp4_weight(55, 0, n, k)
+    x = amax_trap_rows(m, k)
+    W, S, g = dev_weight(w)
+    y = bits(nv.gemv(W, S, g, dev_x(x)))
+    torch.cuda.synchronize()
+    assert np.isfinite(oracle.bf16_value(y)).all()
+    ref, a = oracle.gemv(w.packed, w.scales, w.g, x)
+    check_single(y, ref, a, f"row maximum in a low half, M={m}")
+    y1 = bits(nv.gemv(W, S, g, dev_x(x[:1])))
+    torch.cuda.synchronize()
+    assert np.array_equal(y1[0], y[m - 1])
+
+
+def test_row_maximum_in_a_low_half_word_on_the_tier():
+    n, k, m = 1000, 5120, 16
+    w = synth.nvfp4_weight(56, 0, n, k)
+    x = amax_trap_rows(m, k)
+    W, S, g = dev_weight(w)
+    y = bits(nv.gemv(W, S, g, dev_x(x), wide_tensor=True))
+    torch.cuda.synchronize()
+    assert np.isfinite(oracle.bf16_value(y)).all()
+    ref, a = oracle.gemv(w.packed, w.scales, w.g, x)
+    check_single(y, ref, a, "row maximum in a low half, tier")

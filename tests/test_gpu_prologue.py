@@ -324,3 +324,54 @@ def test_prologue_with_multi_on_the_tier():
         rows = sample_rows(w.n, 100) if w.n > 2048 else None
         check_pro_single(ys[o] if rows is None else ys[o][:, rows], w, xn, near,
                          f"multi tier output {o}", rows)
+
+
+def gated_inputs(seed, m, k, g):
+    x = synth.normal_f32(seed, 400_000_000, m * k, 1.0).reshape(m, k)
+    z = synth.gate_logits(seed, 410_000_000, m, k)
+    gamma = synth.norm_gains(seed, 420_000_000, g)
+    return x, z, gamma
+
+
+def dev_f32(a):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
+
+
+@pytest.mark.parametrize("m", [1, 8, 19])
+def test_gated_rmsnorm_single(m):
+    # the GatedDeltaNet's output projection: K = 48 heads x 128 channels, fp32 x
+    n, k, g, eps = 2000, 6144, 128, 1e-6
+    w = synth.nvfp4_weight(52, 0, n, k)
+    x, z, gamma = gated_inputs(52, m, k, g)
+    W, S, gs = dev_weight(w)
+    y = bits(nv.gemv(W, S, gs, dev_f32(x), prologue=nv.GatedRmsNorm(dev_x(z), dev_vec(gamma), g,
+                                                                     eps)))
+    xo, near = oracle.gated_rmsnorm(x, z, gamma, g, eps)
+    check_pro_single(y, w, xo, near, f"gated rmsnorm M={m}")
+    r = m - 1
+    y1 = bits(nv.gemv(W, S, gs, dev_f32(x[r:r + 1]),
+                      prologue=nv.GatedRmsNorm(dev_x(z[r:r + 1]), dev_vec(gamma), g, eps)))
+    assert np.array_equal(y1[0], y[r]), f"row {r}"
+
+
+@pytest.mark.parametrize("g", [256, 512])
+def test_gated_rmsnorm_group_sizes(g):
+    n, k, m, eps = 700, 2048, 3, 1e-5
+    w = synth.nvfp4_weight(53, 0, n, k)
+    x, z, gamma = gated_inputs(53, m, k, g)
+    W, S, gs = dev_weight(w)
+    y = bits(nv.gemv(W, S, gs, dev_f32(x), prologue=nv.GatedRmsNorm(dev_x(z), dev_vec(gamma), g,
+                                                                     eps)))
+    xo, near = oracle.gated_rmsnorm(x, z, gamma, g, eps)
+    check_pro_single(y, w, xo, near, f"gated rmsnorm G={g}")
+
+
+def test_gated_rmsnorm_ignores_the_wide_flag():
+    n, k, m, g = 1024, 5120, 24, 128
+    w = synth.nvfp4_weight(54, 0, n, k)
+    x, z, gamma = gated_inputs(54, m, k, g)
+    W, S, gs = dev_weight(w)
+    pro = nv.GatedRmsNorm(dev_x(z), dev_vec(gamma), g)
+    y_wide = bits(nv.gemv(W, S, gs, dev_f32(x), prologue=pro, wide_tensor=True))
+    y_pass = bits(nv.gemv(W, S, gs, dev_f32(x), prologue=pro))
+    assert np.array_equal(y_wide, y_pass)
