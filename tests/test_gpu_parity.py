@@ -388,3 +388,42 @@ def test_row_maximum_in_a_low_half_word_on_the_tier():
     assert np.isfinite(oracle.bf16_value(y)).all()
     ref, a = oracle.gemv(w.packed, w.scales, w.g, x)
     check_single(y, ref, a, "row maximum in a low half, tier")
+
+
+def heavy_tailed_rows(seed, m, k):
+    """x rows of N(0, 1) draws times e^N(0, 3^2): magnitudes spread over ~30 binades, the shape
+    of a gated activation; the largest values of a row are far from the next ones."""
+    a = synth.normal_f32(seed, 0, m * k, 1.0).astype(np.float64)
+    s = synth.normal_f32(seed, 2 * m * k, m * k, 3.0).astype(np.float64)
+    return oracle.bf16_rne((a * np.exp(s)).reshape(m, k))
+
+
+def test_heavy_tailed_rows_on_every_path():
+    n, k = 1000, 5120
+    w = synth.nvfp4_weight(57, 0, n, k)
+    wu = synth.nvfp4_weight(57, 10_000_000, n, k)
+    W, S, g = dev_weight(w)
+    Wu, Su, gu = dev_weight(wu)
+    for m, wide in ((8, False), (19, False), (24, True)):
+        x = heavy_tailed_rows(57 + m, m, k)
+        ref, a = oracle.gemv(w.packed, w.scales, w.g, x)
+        y = bits(nv.gemv(W, S, g, dev_x(x), wide_tensor=wide))
+        torch.cuda.synchronize()
+        check_single(y, ref, a, f"heavy tails, single, M={m}, tier={wide}")
+        o = bits(nv.gemv_dual(W, S, g, Wu, Su, gu, dev_x(x), wide_tensor=wide))
+        torch.cuda.synchronize()
+        o_ref, yg, yu, ag, au = oracle.gemv_dual(w.packed, w.scales, w.g, wu.packed, wu.scales,
+                                                 wu.g, x)
+        check_dual(o, o_ref, yg, yu, ag, au, f"heavy tails, dual, M={m}, tier={wide}")
+        # two outputs share one split (not the single call's), so compare with the oracle
+        ys = [bits(t) for t in nv.gemv_multi([(W, S, g), (Wu, Su, gu)], dev_x(x),
+                                             wide_tensor=wide)]
+        torch.cuda.synchronize()
+        check_single(ys[0], ref, a, f"heavy tails, multi output 0, M={m}, tier={wide}")
+        check_single(ys[1], yu, au, f"heavy tails, multi output 1, M={m}, tier={wide}")
+        if not wide:
+            # rows as in calls of their own
+            for r in (0, m - 1):
+                y1 = bits(nv.gemv(W, S, g, dev_x(x[r:r + 1])))
+                torch.cuda.synchronize()
+                assert np.array_equal(y1[0], y[r]), f"row {r} of M={m}"
