@@ -960,12 +960,11 @@ def run_prologue(args, world, rank, local):
             for li in range(n_layers):
                 qkv, o, gu, down = ents[4 * li:4 * li + 4]
                 torch_norm(x, r, gammas[2 * li], hbuf[0], m)
-                fns = [(L.nvfp4_gemv_ex, (qkv["W"].data_ptr(), qkv["S"].data_ptr(),
-                        ctypes.c_float(qkv["g"]), xn_buf.data_ptr(), k_model, qkv["y"].data_ptr(),
-                        qkv["p"].n, m, qkv["p"].n, k_model, wsp, wsn, flags, h))]
-                for fn, a in fns:
-                    if fn(*a) != 0:
-                        raise RuntimeError("launch failed")
+                if L.nvfp4_gemv_ex(qkv["W"].data_ptr(), qkv["S"].data_ptr(),
+                                   ctypes.c_float(qkv["g"]), xn_buf.data_ptr(), k_model,
+                                   qkv["y"].data_ptr(), qkv["p"].n, m, qkv["p"].n, k_model, wsp,
+                                   wsn, flags, h) != 0:
+                    raise RuntimeError("launch failed")
                 xg_buf[:m].copy_((attn[li][:m].float() * torch.sigmoid(gates[li][:m].float()))
                                  .to(torch.bfloat16))
                 if L.nvfp4_gemv_ex(o["W"].data_ptr(), o["S"].data_ptr(), ctypes.c_float(o["g"]),
@@ -1213,7 +1212,6 @@ def run_wide(args, world, rank, local):
     for mode, flags in (("passes", nv.FLAG_PREFETCH_WEIGHTS), ("tensor_tier", nv.FLAG_WIDE_TENSOR)):
         per_mode[mode] = run_wide_mode(args, world, L, ents, ws, stream, flags,
                                        ClockSampler(local) if mode == "tensor_tier" else None)
-    peak, peak_src = peaks()
     top = per_mode["tensor_tier"][WIDE_ROWS[-1]]
     m = WIDE_ROWS[-1]
 
