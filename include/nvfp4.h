@@ -240,10 +240,12 @@ typedef struct {
  * overlap x, residual, gamma or any y, and residual may not overlap y: NVFP4_ERR_ALIAS (the
  * prologue may read x and the residual again after writing h, and y is written after it; so
  * the residual is not updated in place).  With NVFP4_FLAG_WIDE_TENSOR the tier's x pass
- * applies the same prologue, and its rows are invariant over 9..128 as without one.
+ * applies the residual add + RMS norm and the sigmoid gate itself, and its rows are invariant
+ * over 9..128 as without one.
  * Errors: those of the call without a prologue, and NVFP4_ERR_SHAPE (unknown kind, eps
- * negative or not finite, a leading dimension < K), NVFP4_ERR_NULL (a required array NULL when
- * K > 0), NVFP4_ERR_ALIGN, NVFP4_ERR_ALIAS, all checked before anything is enqueued. */
+ * negative or not finite, a leading dimension < K, a group size out of range or not dividing
+ * K), NVFP4_ERR_NULL (a required array NULL when K > 0), NVFP4_ERR_ALIGN, NVFP4_ERR_ALIAS, all
+ * checked before anything is enqueued. */
 int nvfp4_gemv_pro(const nvfp4_prologue_t* prologue, const uint8_t* w, const uint8_t* s,
                    float global_scale, const void* x, int64_t ldx, void* y, int64_t ldy, int m,
                    int64_t n, int64_t k, void* workspace, size_t workspace_bytes, uint32_t flags,
