@@ -52,3 +52,32 @@ def test_reference_arm_runs_on_rank_zero_only():
         steps, warmup = 1, 0
     # a non-zero rank leaves without building the workload or touching the oracle
     assert bench.run_reference(Args(), 2, 1) is None
+
+
+def test_reference_arm_line_at_rank_zero(monkeypatch):
+    # the reference arm's JSON line on the 256 x 512 workload: the oracle timed on host cores,
+    # with the keys the benchmark contract asks of that arm
+    monkeypatch.setattr(bench, "WORKLOAD", "tiny")
+
+    class Args:
+        steps, warmup = 2, 1
+    line = bench.run_reference(Args(), 1, 0)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config"):
+        assert key in line, key
+    assert line["impl"] == "reference"
+    assert (line["steps"], line["warmup"], line["n_gpus"]) == (2, 1, 1)
+    assert line["value"] > 0 and line["ms_per_step"] > 0 and line["higher_is_better"] is True
+    cpu = line["cpu_baseline"]
+    assert cpu["kind"] == "oracle" and cpu["value"] == line["value"] and cpu["cores"] >= 1
+    assert cpu["unit"] == line["unit"] == line["e2e"]["unit"]
+    assert line["e2e"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_cpu_baseline_sample_is_bounded():
+    import synth
+    wl = synth.make("tiny")
+    cpu = bench.cpu_oracle_sample(wl, 0.2)
+    assert cpu["kind"] == "oracle" and cpu["unit"] == "GB/s" and cpu["cores"] >= 1
+    assert cpu["value"] > 0 and "256 consecutive output rows" in cpu["sample"]
