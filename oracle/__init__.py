@@ -97,7 +97,9 @@ def e4m3_table() -> np.ndarray:
 def bf16_value(bits) -> np.ndarray:
     """bf16 bit patterns -> fp64 values (vectorised)."""
     b = np.asarray(bits, np.uint16)
-    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    # widening a signalling-NaN pattern raises the invalid flag; the result is a NaN either way
+    with np.errstate(invalid="ignore"):
+        return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def bf16_rne(values) -> np.ndarray:
