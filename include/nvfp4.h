@@ -42,10 +42,15 @@
  *   - Errors are returned as nvfp4_status codes (never exceptions or aborts).  Argument
  *     checks run on the host before any CUDA call.
  *   - The workspace (nvfp4_workspace_bytes) must be zero-filled before its first use.  It
- *     holds an error word, one completion flag per CTA and fp32 partial sums; every call
- *     that completes resets the flags to zero, so the same workspace serves any number of
- *     calls in stream order (and CUDA-graph replays) without re-zeroing.  Calls that may run
- *     concurrently (different streams) need different workspaces.
+ *     holds an error word, one hand-off word per CTA and fp32 partial sums: the persistent grid
+ *     splits a weight's 128-row groups over the GPU's SMs, and a group cut between CTAs is
+ *     finished by the CTA holding its first unit, which adds the others' partial sums in a fixed
+ *     order.  That CTA waits for them at most 50 us; if they are not resident yet (other work
+ *     holds SMs) it hands the group over and the last of them finishes it, so a call needs no
+ *     co-residency of its CTAs and no wait is unbounded.  Every call that completes resets the
+ *     words to zero, so the same workspace serves any number of calls in stream order (and
+ *     CUDA-graph replays) without re-zeroing: the library is stateless per workspace, not per
+ *     call.  Calls that may run concurrently (different streams) need different workspaces.
  */
 #ifndef NVFP4_H
 #define NVFP4_H
@@ -267,17 +272,19 @@ int nvfp4_gemv_multi_pro(const nvfp4_prologue_t* prologue, const nvfp4_output_t*
  * (cudaMalloc there would take memory outside that budget and synchronise the device).
  *
  * Arguments, layout, guarantees and results are those of nvfp4_gemv with flags 0; the
- * workspace is replaced by a scratch array compiled into this library (2,622,464 bytes of
- * device memory on each device that loads it: an error word, one flag per CTA and one pair of
- * fp32 partial tiles per CTA, for grids of up to 160 CTAs).  The call allocates nothing.
+ * workspace is replaced by a scratch array compiled into this library (2,622,720 bytes of
+ * device memory on each device that loads it: an error word, one hand-off word per CTA and two
+ * pairs of fp32 partial tiles per CTA, for grids of up to 160 CTAs).  The call allocates
+ * nothing.
  *
- * Set-up: the first call on a device (made, like every call, with that device current) looks
- * up the array's device address with cudaGetSymbolAddress; make that first call before any
- * stream capture.  NVFP4_ERR_LAUNCH if the lookup fails.
+ * Set-up: every call (made with the intended device current) looks up the array's device
+ * address in the current context with cudaGetSymbolAddress, a host-side lookup that allocates
+ * nothing; the first call on a device may also load the library's module there, so make that
+ * first call before any stream capture.  NVFP4_ERR_LAUNCH if the lookup fails.
  *
  * Sharing: every call on a device uses the same array and finds it as the previous call left
- * it.  Each call therefore first clears the error word and the flags (a cudaMemsetAsync of the
- * first 1,024 bytes on `stream`), then launches.  Calls that overlap in time -- on different
+ * it.  Each call therefore first clears the error word and the hand-off words (a
+ * cudaMemsetAsync of the first 1,280 bytes on `stream` on a 148-SM B200), then launches.  Calls that overlap in time -- on different
  * streams, or from different host threads -- race on the array and give wrong results:
  * issue them in one stream's order.  If a bounded wait inside the kernel gives up, the kernel
  * records it in the array's error word, which this call cannot report; callers that need
@@ -289,6 +296,75 @@ int nvfp4_gemv_noalloc(const uint8_t* w, const uint8_t* s, float global_scale, c
                        int64_t ldx, void* y, int64_t ldy, int m, int64_t n, int64_t k,
                        cudaStream_t stream);
 
+/* Chains: up to NVFP4_CHAIN_MAX_OPS GEMV operations in one persistent launch, run in order,
+ * an operation optionally reading an earlier one's result as its x.  The decode plan runs its
+ * projections as separate launches ("Blueprint - circuit executor" page, table "Kernels the
+ * plan launches": w4a16_gemv_dual x64 feeding w4a16_gemv_sw, the MLP's gate_up and down); a
+ * launch's fixed start and drain then cost more HBM time than a small projection streams.  In
+ * a chain the weight stream continues across the boundaries: while one operation finishes,
+ * the next one's weights already stream into shared memory (they do not depend on earlier
+ * results).  An operation with x_from >= 0 waits on the device, per CTA, until every row group
+ * of that earlier operation is written, then reads it.
+ *
+ * Every operation's result is bitwise that of the same call made alone (nvfp4_gemv_multi for
+ * NVFP4_OP_SINGLE, nvfp4_gemv_dual for NVFP4_OP_DUAL, on the same x): each keeps its own work
+ * split.  Row invariance over M = 1..128 and determinism therefore hold as for those calls.
+ */
+#define NVFP4_CHAIN_MAX_OPS 16
+#define NVFP4_OP_SINGLE 0 /* 1..NVFP4_MAX_OUTPUTS weights sharing x (nvfp4_gemv_multi) */
+#define NVFP4_OP_DUAL 1   /* silu(gate x) * (up x) (nvfp4_gemv_dual) */
+
+typedef struct {
+    int32_t kind;    /* NVFP4_OP_SINGLE or NVFP4_OP_DUAL */
+    int32_t outputs; /* NVFP4_OP_SINGLE: 1..NVFP4_MAX_OUTPUTS; NVFP4_OP_DUAL: 1 */
+    /* NVFP4_OP_SINGLE: the outputs, each N >= 1.  NVFP4_OP_DUAL: out[0] is the gate weight and
+     * the result o (y, ldy, n), out[1] the up weight (its n must equal out[0].n; its y and ldy
+     * are ignored). */
+    nvfp4_output_t out[NVFP4_MAX_OUTPUTS];
+    const void* x;   /* bf16 [M][ldx], used when x_from < 0 */
+    int64_t ldx;
+    int64_t k;       /* K of every weight of the operation: K % 256 == 0 */
+    int32_t x_from;  /* -1: x as given.  j in [0, this operation's index): x is operation j's
+                        result (j must have one output, with n == this K, y 16-byte aligned
+                        and ldy % 8 == 0; x and ldx are then ignored) */
+} nvfp4_chain_op_t;
+
+/* Workspace bytes of nvfp4_gemv_chain for these operations and M (host only, besides the
+ * device's SM count): a header and, per kernel operation, one arrival count and two partial
+ * tiles (per weight stream) per SM -- about 1.2 MB per single operation and 2.4 MB per dual on
+ * a 148-SM B200.  Errors as nvfp4_gemv_chain's argument checks, and NVFP4_ERR_ARCH. */
+int nvfp4_chain_workspace_bytes(const nvfp4_chain_op_t* ops, int count, int m, size_t* bytes);
+
+/* Runs `count` (1..NVFP4_CHAIN_MAX_OPS) operations in order, M (1..128) rows each, one kernel
+ * launch per 8-row pass.  ops is host memory read during the call only.  Per operation, the
+ * rules of nvfp4_gemv_multi / nvfp4_gemv_dual hold, plus: K % 256 == 0 and every scale array
+ * 16-byte aligned (the scale codes move by TMA).  An operation whose row groups exceed one
+ * launch at its K (only for K above 9,728 with more than 10,496 rows) is cut into row chunks
+ * as nvfp4_gemv cuts it; the chain may then hold at most NVFP4_CHAIN_MAX_OPS chunks in all.
+ * Outputs may not overlap one another, any x or any weight: operations run concurrently on
+ * different SMs, ordered only through x_from.
+ *   workspace: 16-byte aligned, nvfp4_chain_workspace_bytes(ops, count, m) bytes, zero-filled
+ *     before first use; reset by every completed launch, as for nvfp4_gemv.
+ *   flags: 0 or NVFP4_FLAG_PREFETCH_WEIGHTS (the chain's first weights stream in while the
+ *     kernel before it finishes).
+ * A chain with x_from links is launched cooperatively (all CTAs resident at once), so its
+ * waits always end; each wait still gives up after 1 s and then sets the workspace's error word
+ * to 4 (results invalid; nvfp4_workspace_error reads it).
+ * Errors: NVFP4_ERR_NULL, NVFP4_ERR_SHAPE (count, kind, outputs, K, x_from out of range or its
+ * source not one output of N == K, too many chunks, unknown flags), NVFP4_ERR_ROWS,
+ * NVFP4_ERR_ALIGN, NVFP4_ERR_WORKSPACE, NVFP4_ERR_ARCH, NVFP4_ERR_LAUNCH; all checked before
+ * anything is enqueued. */
+int nvfp4_gemv_chain(const nvfp4_chain_op_t* ops, int count, int m, void* workspace,
+                     size_t workspace_bytes, uint32_t flags, cudaStream_t stream);
+
+/* Test form of nvfp4_gemv_chain, for the bounded waits: the first operation that a later one
+ * reads never reports its completion, and the waits give up after wait_limit_ns (1 .. 1e9).
+ * The launch then ends normally with error word 4 in the workspace and that reader's outputs
+ * invalid; the device stays usable.  No other use. */
+int nvfp4_gemv_chain_unsignalled(const nvfp4_chain_op_t* ops, int count, int m, void* workspace,
+                                 size_t workspace_bytes, int64_t wait_limit_ns,
+                                 cudaStream_t stream);
+
 /* Workspace bytes of an nvfp4_gemv_ex / _pro, nvfp4_gemv_dual_ex / _pro or nvfp4_gemv_multi /
  * _pro (the largest of its outputs' sizes) call of M rows with
  * NVFP4_FLAG_WIDE_TENSOR or an input prologue: the nvfp4_workspace_bytes layout followed by the
@@ -299,8 +375,9 @@ int nvfp4_gemv_noalloc(const uint8_t* w, const uint8_t* s, float global_scale, c
 int nvfp4_workspace_bytes_wide(int64_t n, int64_t k, int m, size_t* bytes);
 
 /* The workspace's error word after the work enqueued so far has run (synchronises the
- * stream): 0 if no kernel hit a bounded wait's limit, else a nonzero code (results of the
- * call that set it are then invalid; zero-fill the workspace before reuse).
+ * stream): 0 if no kernel hit a bounded wait's limit, else a nonzero code -- 2 or 3: a wait on
+ * the shared-memory ring (a weight copy that never landed), 4: a chain's dependency wait --
+ * and the results of the call that set it are invalid (zero-fill the workspace before reuse).
  * Returns NVFP4_OK and writes *error, or an nvfp4_status error. */
 int nvfp4_workspace_error(const void* workspace, size_t workspace_bytes, cudaStream_t stream,
                           int32_t* error);

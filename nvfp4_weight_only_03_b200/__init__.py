@@ -9,6 +9,8 @@ missing or the device is not a B200 the calls raise.
     o = gemv_dual(wg, sg, gg, wu, su, gu, x)  # o = bf16(silu(gate) * up)
     k_, v_ = gemv_multi([(wk, sk, gk), (wv, sv, gv)], x)  # several outputs sharing x, one pass
     q = gemv(w, s, g, x, prologue=AddRmsNorm(r, gamma, 1e-6, h))  # x' = rmsnorm(x + r) first
+    o, d = gemv_chain([ChainOp.dual(wg, sg, gg, wu, su, gu, x=x),    # one launch: gate_up ...
+                       ChainOp.single([(wd, sd, gd)], x_from=0)])   # ... feeding down
 
 w: uint8 [N][K/2] packed e2m1 (low nibble = even k), s: uint8 [N][K/16] e4m3 scale codes,
 g: float global scale, x: bfloat16 [M][K] (M = 1..128, one kernel pass per 8 rows; row stride
@@ -35,6 +37,8 @@ MAX_OUTPUTS = 4
 GROUP = 16
 FLAG_PREFETCH_WEIGHTS = 1
 FLAG_WIDE_TENSOR = 2
+CHAIN_MAX_OPS = 16
+OP_SINGLE, OP_DUAL = 0, 1
 
 
 class Nvfp4Error(RuntimeError):
@@ -47,6 +51,13 @@ class Output(ctypes.Structure):
     """nvfp4_output_t: one output of nvfp4_gemv_multi."""
     _fields_ = [("w", ctypes.c_void_p), ("s", ctypes.c_void_p), ("global_scale", ctypes.c_float),
                 ("y", ctypes.c_void_p), ("ldy", ctypes.c_int64), ("n", ctypes.c_int64)]
+
+
+class ChainOpStruct(ctypes.Structure):
+    """nvfp4_chain_op_t: one operation of nvfp4_gemv_chain."""
+    _fields_ = [("kind", ctypes.c_int32), ("outputs", ctypes.c_int32),
+                ("out", Output * MAX_OUTPUTS), ("x", ctypes.c_void_p), ("ldx", ctypes.c_int64),
+                ("k", ctypes.c_int64), ("x_from", ctypes.c_int32)]
 
 
 class Prologue(ctypes.Structure):
@@ -164,12 +175,18 @@ def lib():
         L.nvfp4_gemv_multi_pro.argtypes = [pp] + L.nvfp4_gemv_multi.argtypes
         L.nvfp4_workspace_error.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
         L.nvfp4_workspace_bytes_wide.argtypes = [i64, i64, c_int, ctypes.POINTER(sz)]
+        cp = ctypes.POINTER(ChainOpStruct)
+        L.nvfp4_chain_workspace_bytes.argtypes = [cp, c_int, c_int, ctypes.POINTER(sz)]
+        L.nvfp4_gemv_chain.argtypes = [cp, c_int, c_int, vp, sz, ctypes.c_uint32, vp]
+        L.nvfp4_gemv_chain_unsignalled.argtypes = [cp, c_int, c_int, vp, sz, i64, vp]
         L.nvfp4_status_string.argtypes = [c_int]
         L.nvfp4_status_string.restype = ctypes.c_char_p
         for f in (L.nvfp4_pack_info, L.nvfp4_workspace_bytes, L.nvfp4_gemv, L.nvfp4_gemv_dual,
                   L.nvfp4_gemv_ex, L.nvfp4_gemv_dual_ex, L.nvfp4_gemv_noalloc,
                   L.nvfp4_gemv_multi, L.nvfp4_workspace_error, L.nvfp4_workspace_bytes_wide,
-                  L.nvfp4_gemv_pro, L.nvfp4_gemv_dual_pro, L.nvfp4_gemv_multi_pro):
+                  L.nvfp4_gemv_pro, L.nvfp4_gemv_dual_pro, L.nvfp4_gemv_multi_pro,
+                  L.nvfp4_chain_workspace_bytes, L.nvfp4_gemv_chain,
+                  L.nvfp4_gemv_chain_unsignalled):
             f.restype = c_int
         _lib = L
     return _lib
@@ -198,20 +215,46 @@ def workspace_bytes_wide(n: int, k: int, m: int) -> int:
     return int(b.value)
 
 
+# Default workspaces, one per (device, stream, kind): calls on different streams may run at
+# the same time, and two calls sharing a workspace at the same time would mix their arrival
+# counts and partial sums.  Calls on one stream run in order, so they share one.  The cache
+# keeps a reference to each torch stream, so its handle cannot be reused by a new stream while
+# the workspace is in the cache.
 _workspaces: dict = {}
 
 
-def workspace(device=None) -> torch.Tensor:
-    """A zero-filled workspace for `device` (cached; one per device, for the default use of
-    one stream at a time)."""
-    dev = torch.device("cuda", torch.cuda.current_device() if device is None else
-                       torch.device(device).index or 0)
-    ws = _workspaces.get(dev)
-    if ws is None:
-        with torch.cuda.device(dev):
-            ws = torch.zeros(workspace_bytes(), dtype=torch.uint8, device=dev)
-        _workspaces[dev] = ws
-    return ws
+def _device_of(device) -> torch.device:
+    return torch.device("cuda", torch.cuda.current_device() if device is None else
+                        torch.device(device).index or 0)
+
+
+def _stream_obj(stream, dev):
+    if stream is None:
+        return torch.cuda.current_stream(dev)
+    if hasattr(stream, "cuda_stream"):
+        return stream
+    return torch.cuda.ExternalStream(int(stream), device=dev)
+
+
+def _cached_workspace(kind: str, need: int, device, stream) -> torch.Tensor:
+    dev = _device_of(device)
+    st = _stream_obj(stream, dev)
+    key = (dev, st.cuda_stream, kind)
+    ent = _workspaces.get(key)
+    if ent is None or ent[0].numel() < need:
+        # allocated (and zero-filled) on the stream that uses it: when a grown workspace
+        # replaces it, the caching allocator reuses the old block only in that stream's order
+        with torch.cuda.device(dev), torch.cuda.stream(st):
+            ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+        ent = (ws, st)
+        _workspaces[key] = ent
+    return ent[0]
+
+
+def workspace(device=None, stream=None) -> torch.Tensor:
+    """The zero-filled default workspace of (device, stream): cached, one per stream, so calls
+    on different streams never share one."""
+    return _cached_workspace("plain", workspace_bytes(), device, stream)
 
 
 def workspace_error(ws: torch.Tensor, stream=None) -> int:
@@ -257,26 +300,24 @@ def _out(y, m, n, x):
     return y, y.stride(0) if m > 1 else n
 
 
-_wide_workspaces: dict = {}
+def wide_workspace(n: int, k: int, m: int, device=None, stream=None) -> torch.Tensor:
+    """The default workspace of (device, stream) for a wide_tensor or prologue call of this
+    shape (grown when a larger one is needed)."""
+    return _cached_workspace("wide", workspace_bytes_wide(n, k, m), device, stream)
 
 
-def wide_workspace(n: int, k: int, m: int, device=None) -> torch.Tensor:
-    """A zero-filled workspace large enough for a wide_tensor call of this shape (cached per
-    device, grown when a larger one is needed)."""
-    dev = torch.device("cuda", torch.cuda.current_device() if device is None else
-                       torch.device(device).index or 0)
-    need = workspace_bytes_wide(n, k, m)
-    ws = _wide_workspaces.get(dev)
-    if ws is None or ws.numel() < need:
-        with torch.cuda.device(dev):
-            ws = torch.zeros(need, dtype=torch.uint8, device=dev)
-        _wide_workspaces[dev] = ws
-    return ws
+def _check_error(ws: torch.Tensor, stream, where: str):
+    """Opt-in check after a call: synchronises the stream and raises if a bounded wait in the
+    call's kernels gave up (the results are then invalid)."""
+    err = workspace_error(ws, stream)
+    if err != 0:
+        raise RuntimeError(f"{where}: a bounded wait gave up (workspace error word {err}); "
+                           "the results are invalid")
 
 
 def gemv(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor, y: torch.Tensor = None,
          ws: torch.Tensor = None, stream=None, prefetch_weights: bool = False,
-         wide_tensor: bool = False, prologue=None) -> torch.Tensor:
+         wide_tensor: bool = False, prologue=None, check: bool = False) -> torch.Tensor:
     """y[m][n] = bf16(g * sum_k e2m1(w[n][k]) * e4m3(s[n][k/16]) * x[m][k]) on the GPU.
 
     prefetch_weights: stream w and s before earlier work on the stream has finished
@@ -284,13 +325,16 @@ def gemv(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor, y: torch.T
     wide_tensor: calls of 9..128 rows run on the tensor-core tier (one pass over the weights;
     rows invariant over 9..128, equal to 1..8-row calls within the tolerance).
     prologue: AddRmsNorm or SigmoidGate, applied to x inside the call (its x' lives in the
-    workspace, so a caller's ws must hold workspace_bytes_wide(n, k, m))."""
+    workspace, so a caller's ws must hold workspace_bytes_wide(n, k, m)).
+    ws: the workspace; by default the cached one of (x's device, stream).
+    check: synchronise after the call and raise if a bounded wait in its kernels gave up."""
     n, k = _weight_args(w, s)
     x, m, ldx = _x_args(x, k, getattr(prologue, "x_dtype", torch.bfloat16))
     pro = None if prologue is None else prologue.struct(m, k)
     y, ldy = _out(y, m, n, x)
     if ws is None:
-        ws = wide_workspace(n, k, m, x.device) if (wide_tensor or pro) else workspace(x.device)
+        ws = wide_workspace(n, k, m, x.device, stream) if (wide_tensor or pro) else \
+            workspace(x.device, stream)
     flags = (FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0) | \
         (FLAG_WIDE_TENSOR if wide_tensor else 0)
     args = (w.data_ptr(), s.data_ptr(), float(g), x.data_ptr(), ldx, y.data_ptr(), ldy, m, n, k,
@@ -300,6 +344,8 @@ def gemv(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor, y: torch.T
     else:
         st = lib().nvfp4_gemv_pro(ctypes.byref(pro), *args)
     _check(st, "nvfp4_gemv")
+    if check:
+        _check_error(ws, stream, "nvfp4_gemv")
     return y
 
 
@@ -320,11 +366,11 @@ def gemv_noalloc(w: torch.Tensor, s: torch.Tensor, g: float, x: torch.Tensor,
 def gemv_dual(wg: torch.Tensor, sg: torch.Tensor, gg: float, wu: torch.Tensor, su: torch.Tensor,
               gu: float, x: torch.Tensor, y: torch.Tensor = None, ws: torch.Tensor = None,
               stream=None, prefetch_weights: bool = False,
-              wide_tensor: bool = False, prologue=None) -> torch.Tensor:
+              wide_tensor: bool = False, prologue=None, check: bool = False) -> torch.Tensor:
     """o[m][n] = bf16(silu(gate) * up), gate/up the two NVFP4 GEMVs of the same x.
 
     wide_tensor: calls of 9..128 rows run gate and up on the tensor-core tier, kept in fp32
-    and combined by one final pass.  prologue: as for gemv."""
+    and combined by one final pass.  prologue, ws, check: as for gemv."""
     n, k = _weight_args(wg, sg)
     if _weight_args(wu, su) != (n, k):
         raise ValueError("gate and up weights must have the same shape")
@@ -332,7 +378,8 @@ def gemv_dual(wg: torch.Tensor, sg: torch.Tensor, gg: float, wu: torch.Tensor, s
     pro = None if prologue is None else prologue.struct(m, k)
     y, ldy = _out(y, m, n, x)
     if ws is None:
-        ws = wide_workspace(n, k, m, x.device) if (wide_tensor or pro) else workspace(x.device)
+        ws = wide_workspace(n, k, m, x.device, stream) if (wide_tensor or pro) else \
+            workspace(x.device, stream)
     flags = (FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0) | \
         (FLAG_WIDE_TENSOR if wide_tensor else 0)
     args = (wg.data_ptr(), sg.data_ptr(), float(gg), wu.data_ptr(), su.data_ptr(), float(gu),
@@ -343,16 +390,20 @@ def gemv_dual(wg: torch.Tensor, sg: torch.Tensor, gg: float, wu: torch.Tensor, s
     else:
         st = lib().nvfp4_gemv_dual_pro(ctypes.byref(pro), *args)
     _check(st, "nvfp4_gemv_dual")
+    if check:
+        _check_error(ws, stream, "nvfp4_gemv_dual")
     return y
 
 
 def gemv_multi(weights, x: torch.Tensor, ys=None, ws: torch.Tensor = None, stream=None,
-               prefetch_weights: bool = False, prologue=None, wide_tensor: bool = False) -> list:
+               prefetch_weights: bool = False, prologue=None, wide_tensor: bool = False,
+               check: bool = False) -> list:
     """Several GEMVs sharing x in one pass (nvfp4_gemv_multi): weights is a list of up to
     MAX_OUTPUTS (w, s, g) triples with the same K; returns [y_0, y_1, ...], y_o the GEMV of
     weight o as gemv computes it.  ys: optional preallocated outputs, one per weight.
     prologue: as for gemv, applied once to the shared x.  wide_tensor: 9..128 rows on the
-    tensor-core tier, each output bitwise as gemv(..., wide_tensor=True) computes it."""
+    tensor-core tier, each output bitwise as gemv(..., wide_tensor=True) computes it.
+    ws, check: as for gemv."""
     weights = list(weights)
     if not 1 <= len(weights) <= MAX_OUTPUTS:
         raise ValueError(f"1..{MAX_OUTPUTS} weights, got {len(weights)}")
@@ -375,9 +426,9 @@ def gemv_multi(weights, x: torch.Tensor, ys=None, ws: torch.Tensor = None, strea
     if ws is None:
         if pro is not None or wide_tensor:
             ws = wide_workspace(max(shapes, key=lambda nk: workspace_bytes_wide(nk[0], k, m))[0],
-                                k, m, x.device)
+                                k, m, x.device, stream)
         else:
-            ws = workspace(x.device)
+            ws = workspace(x.device, stream)
     flags = (FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0) | \
         (FLAG_WIDE_TENSOR if wide_tensor else 0)
     args = (outs, len(weights), x.data_ptr(), ldx, m, k, ws.data_ptr(), ws.numel(), flags,
@@ -387,4 +438,107 @@ def gemv_multi(weights, x: torch.Tensor, ys=None, ws: torch.Tensor = None, strea
     else:
         st = lib().nvfp4_gemv_multi_pro(ctypes.byref(pro), *args)
     _check(st, "nvfp4_gemv_multi")
+    if check:
+        _check_error(ws, stream, "nvfp4_gemv_multi")
     return result
+
+
+class ChainOp:
+    """One operation of gemv_chain: NVFP4 weights sharing an x, which is either a bf16 tensor
+    or the result of an earlier operation of the chain (x_from = its index)."""
+
+    def __init__(self, kind, weights, x=None, x_from=None, ys=None):
+        if (x is None) == (x_from is None):
+            raise ValueError("give exactly one of x and x_from")
+        self.kind, self.weights, self.x, self.x_from = kind, list(weights), x, x_from
+        self.ys = ys
+
+    @classmethod
+    def single(cls, weights, x=None, x_from=None, ys=None):
+        """1..MAX_OUTPUTS (w, s, g) weights sharing x (as gemv_multi)."""
+        return cls(OP_SINGLE, weights, x, x_from, ys)
+
+    @classmethod
+    def dual(cls, wg, sg, gg, wu, su, gu, x=None, x_from=None, y=None):
+        """o = silu(gate x) * (up x) (as gemv_dual)."""
+        return cls(OP_DUAL, [(wg, sg, gg), (wu, su, gu)], x, x_from, None if y is None else [y])
+
+
+def _chain_structs(ops, m_hint=None):
+    """Marshals a list of ChainOp into nvfp4_chain_op_t structs and allocates the outputs."""
+    n_ops = len(ops)
+    if not 1 <= n_ops <= CHAIN_MAX_OPS:
+        raise ValueError(f"1..{CHAIN_MAX_OPS} operations, got {n_ops}")
+    m = m_hint
+    xs = []
+    for op in ops:
+        if op.x is not None:
+            k = _weight_args(*op.weights[0][:2])[1]
+            x, mm, ldx = _x_args(op.x, k)
+            if m is not None and mm != m:
+                raise ValueError("every x of a chain must have the same number of rows")
+            m = mm
+            xs.append((x, ldx))
+        else:
+            xs.append((None, 0))
+    if m is None:
+        raise ValueError("the first operation needs an x")
+    arr = (ChainOpStruct * n_ops)()
+    results, keep = [], []
+    for i, (op, (x, ldx)) in enumerate(zip(ops, xs)):
+        shapes = [_weight_args(w, s) for w, s, _ in op.weights]
+        k = shapes[0][1]
+        if any(kk != k for _, kk in shapes):
+            raise ValueError(f"operation {i}: all weights must have the same K")
+        c = arr[i]
+        c.kind, c.k = op.kind, k
+        c.x_from = -1 if op.x_from is None else int(op.x_from)
+        if x is not None:
+            c.x, c.ldx = x.data_ptr(), ldx
+            keep.append(x)
+        n_out = 1 if op.kind == OP_DUAL else len(op.weights)
+        c.outputs = n_out
+        dev = x.device if x is not None else results[op.x_from][0].device
+        ys = op.ys if op.ys is not None else [None] * n_out
+        outs = []
+        for o in range(n_out):
+            y, ldy = _out(ys[o], m, shapes[o][0], torch.empty(0, device=dev))
+            outs.append(y)
+            c.out[o].y, c.out[o].ldy, c.out[o].n = y.data_ptr(), ldy, shapes[o][0]
+        for j, (w, s, g) in enumerate(op.weights):
+            c.out[j].w, c.out[j].s, c.out[j].global_scale = w.data_ptr(), s.data_ptr(), float(g)
+            if op.kind == OP_DUAL and j == 1:
+                c.out[j].n = shapes[1][0]
+        results.append(outs)
+    return arr, m, results, keep
+
+
+def chain_workspace_bytes(ops, m: int = None) -> int:
+    arr, m, _, _ = _chain_structs(ops, m)
+    b = ctypes.c_size_t()
+    _check(lib().nvfp4_chain_workspace_bytes(arr, len(ops), m, ctypes.byref(b)),
+           "nvfp4_chain_workspace_bytes")
+    return int(b.value)
+
+
+def gemv_chain(ops, ws: torch.Tensor = None, stream=None, prefetch_weights: bool = False,
+               check: bool = False) -> list:
+    """Runs the ChainOp list in one persistent launch per 8-row pass (nvfp4_gemv_chain).
+    Returns, per operation, its output (a tensor) or, for a single operation with several
+    weights, the list of its outputs.  Each is bitwise what gemv_multi / gemv_dual gives for
+    the same x.  ws, check: as for gemv (the default workspace is grown to the chain's size)."""
+    ops = list(ops)
+    arr, m, results, _keep = _chain_structs(ops)
+    b = ctypes.c_size_t()
+    _check(lib().nvfp4_chain_workspace_bytes(arr, len(ops), m, ctypes.byref(b)),
+           "nvfp4_chain_workspace_bytes")
+    dev = results[0][0].device
+    if ws is None:
+        ws = _cached_workspace("chain", int(b.value), dev, stream)
+    st = lib().nvfp4_gemv_chain(arr, len(ops), m, ws.data_ptr(), ws.numel(),
+                                FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0,
+                                _stream(stream))
+    _check(st, "nvfp4_gemv_chain")
+    if check:
+        _check_error(ws, stream, "nvfp4_gemv_chain")
+    return [r[0] if len(r) == 1 else r for r in results]

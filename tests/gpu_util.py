@@ -3,6 +3,11 @@ oracle under the acceptance rules."""
 import numpy as np
 import torch
 
+# One entry per checked call: where, elements, elements more than 1 bf16 ulp from bf16(y_ref)
+# (all of them, near-zero ones included), the largest ulp distance, and the largest error over
+# the tolerance.  conftest.py prints them at the end of the run.
+ULP_RECORDS: list = []
+
 import oracle
 import synth
 import nvfp4_weight_only_03_b200 as nv
@@ -42,11 +47,17 @@ def check_single(y_bits, y_ref, a_ref, where=""):
     worst = int(ulp[strict].max()) if strict.any() else 0
     assert worst <= 1, f"{where}: bf16 ulp distance {worst} on a well-conditioned output"
     err = np.abs(y - y_ref)
-    return {"max_err_over_tol": float((err / tol).max()) if err.size else 0.0,
-            "ulp_gt1_total": int((ulp > 1).sum()), "ulp_max": int(ulp.max()) if ulp.size else 0}
+    res = {"max_err_over_tol": float((err / tol).max()) if err.size else 0.0,
+           "ulp_gt1_total": int((ulp > 1).sum()), "ulp_max": int(ulp.max()) if ulp.size else 0}
+    ULP_RECORDS.append((where or "single", int(ulp.size), res["ulp_gt1_total"], res["ulp_max"],
+                        res["max_err_over_tol"]))
+    return res
 
 
 def check_dual(o_bits, o_ref, yg, yu, ag, au, where=""):
+    """Propagated tolerance on every element, and within 1 bf16 ulp of bf16(o_ref) wherever both
+    pre-activations are well conditioned (each at least 1/16 of its absolute-value sum, as for
+    the single GEMV, and the gate away from zero)."""
     o = oracle.bf16_value(o_bits)
     tol = oracle.dual_tolerance(yg, yu, ag, au, o_ref)
     err = np.abs(o - o_ref)
@@ -55,8 +66,20 @@ def check_dual(o_bits, o_ref, yg, yu, ag, au, where=""):
     ulp = oracle.bf16_ulp_distance(o_bits, oracle.bf16_rne(o_ref))
     well = (np.abs(yg) >= ag / 16) & (np.abs(yu) >= au / 16) & (np.abs(yg) > 1e-3)
     worst = int(ulp[well].max()) if well.any() else 0
-    assert worst <= 2, f"{where}: bf16 ulp distance {worst} on a well-conditioned output"
-    return {"max_err_over_tol": float((err / tol).max()) if err.size else 0.0}
+    assert worst <= 1, f"{where}: bf16 ulp distance {worst} on a well-conditioned output"
+    res = {"max_err_over_tol": float((err / tol).max()) if err.size else 0.0,
+           "ulp_gt1_total": int((ulp > 1).sum()), "ulp_max": int(ulp.max()) if ulp.size else 0}
+    ULP_RECORDS.append((where or "dual", int(ulp.size), res["ulp_gt1_total"], res["ulp_max"],
+                        res["max_err_over_tol"]))
+    return res
+
+
+def assert_ws_clean(ws):
+    """Error word, completion and arrival counts all back at zero after the calls (the partial
+    sums are scratch and may stay): the header's 512 bytes, then one count per SM."""
+    torch.cuda.synchronize()
+    head = ws[:512 + 4 * torch.cuda.get_device_properties(ws.device).multi_processor_count]
+    assert int(head.count_nonzero()) == 0, "workspace counts / error word not left zero"
 
 
 def pack_nibbles(nibs: np.ndarray) -> np.ndarray:

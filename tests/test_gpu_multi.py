@@ -13,7 +13,7 @@ import torch
 import oracle
 import synth
 import nvfp4_weight_only_03_b200 as nv
-from gpu_util import bits, check_single, dev_weight, dev_x
+from gpu_util import assert_ws_clean, bits, check_single, dev_weight, dev_x
 
 pytestmark = pytest.mark.gpu
 
@@ -27,12 +27,6 @@ def multi(weights, x_bits, ws):
     ys = nv.gemv_multi([dev_weight(w) for w in weights], dev_x(x_bits), ws=ws)
     torch.cuda.synchronize()
     return [bits(y) for y in ys]
-
-
-def assert_ws_clean(ws):
-    torch.cuda.synchronize()
-    head = ws[:256 + 4 * torch.cuda.get_device_properties(0).multi_processor_count]
-    assert int(head.count_nonzero()) == 0, "workspace flags / error word not left zero"
 
 
 def check_outputs(weights, x_bits, ys, where, rows=None):

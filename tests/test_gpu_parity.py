@@ -11,8 +11,8 @@ import torch
 import oracle
 import synth
 import nvfp4_weight_only_03_b200 as nv
-from gpu_util import (bits, bf16_bits_of, check_dual, check_single, dev_weight, dev_x,
-                      pack_nibbles, random_weight)
+from gpu_util import (assert_ws_clean, bits, bf16_bits_of, check_dual, check_single, dev_weight,
+                      dev_x, pack_nibbles, random_weight)
 
 pytestmark = pytest.mark.gpu
 
@@ -28,13 +28,6 @@ def run(w, x_bits, ws, m=None):
     y = nv.gemv(W, S, g, dev_x(x_bits[:m]), ws=ws)
     torch.cuda.synchronize()
     return bits(y)
-
-
-def assert_ws_clean(ws):
-    """Error word 0 and every flag reset (partial sums are scratch and may stay)."""
-    torch.cuda.synchronize()
-    head = ws[:256 + 4 * torch.cuda.get_device_properties(0).multi_processor_count]
-    assert int(head.count_nonzero()) == 0, "workspace flags / error word not left zero"
 
 
 # ------------------------------------------------------------------------------------------

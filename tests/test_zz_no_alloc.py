@@ -63,6 +63,24 @@ def test_two_calls_in_a_row_match_the_workspace_path(m):
     assert np.array_equal(first, y_ws) and np.array_equal(second, y_ws)
 
 
+def test_24_rows_run_as_passes_on_the_shared_scratch():
+    # 24 rows: three 8-row kernel passes in stream order, all on the one compiled-in scratch
+    p = synth.make("inproj").projections[0]
+    W, S, g = dev_weight(p.w)
+    n, k = p.w.n, p.w.k
+    rng = np.random.default_rng(24)
+    xb = oracle.bf16_rne(rng.standard_normal((24, k)))
+    x = dev_x(xb)
+    y_ws = bits(with_workspace(W, S, g, x, 24, n, k))
+    first = bits(noalloc(W, S, g, x, 24, n, k))
+    second = bits(noalloc(W, S, g, x, 24, n, k))
+    torch.cuda.synchronize()
+    assert np.array_equal(first, y_ws) and np.array_equal(second, y_ws)
+    rows = np.arange(0, n, 61)
+    ref, a = oracle.gemv(p.w.packed, p.w.scales, p.w.g, xb, rows=rows)
+    check_single(first[:, rows], ref, a, "noalloc M=24 vs oracle (sampled rows)")
+
+
 def test_consecutive_shapes_share_the_scratch():
     # a split-heavy shape, then a small one, then the first again: each call starts from the
     # flags the previous one left and must still be exact
