@@ -330,7 +330,7 @@ typedef struct {
 } nvfp4_chain_op_t;
 
 /* Workspace bytes of nvfp4_gemv_chain for these operations and M (host only, besides the
- * device's SM count): a header and, per kernel operation, one arrival count and two partial
+ * device's SM count): a header and, per kernel operation, one hand-off word and two partial
  * tiles (per weight stream) per SM -- about 1.2 MB per single operation and 2.4 MB per dual on
  * a 148-SM B200.  Errors as nvfp4_gemv_chain's argument checks, and NVFP4_ERR_ARCH. */
 int nvfp4_chain_workspace_bytes(const nvfp4_chain_op_t* ops, int count, int m, size_t* bytes);

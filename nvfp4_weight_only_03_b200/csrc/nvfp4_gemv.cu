@@ -1128,13 +1128,13 @@ int device_info(int* dev_out, DeviceInfo** info) {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Bytes of one kernel operation's arrival counts and partial tiles.
+// Bytes of one kernel operation's hand-off words and partial tiles.
 size_t arrive_bytes(int sms) { return align_up((size_t)sms * 4, 256); }
 size_t partial_bytes(int sms, int streams) {
     return (size_t)sms * 2 * streams * kPartialFloats * sizeof(float);
 }
 
-// Workspace of a single call: the header, then one operation's arrival counts and partial tiles
+// Workspace of a single call: the header, then one operation's hand-off words and partial tiles
 // (sized for two streams, so that every kind of call fits).
 size_t workspace_layout(int sms, size_t* arrive_off, size_t* partial_off) {
     *arrive_off = kHeaderBytes;
@@ -1761,7 +1761,7 @@ int run_chain(const nvfp4_chain_op_t* ops, int count, int m, void* ws, size_t ws
 }  // namespace
 
 // ------------------------------------------------------------------------------------------
-// Scratch of nvfp4_gemv_noalloc: the workspace of nvfp4_gemv (header, one arrival count per CTA,
+// Scratch of nvfp4_gemv_noalloc: the workspace of nvfp4_gemv (header, one hand-off word per CTA,
 // two pairs of partial tiles per CTA, in workspace_layout's order) compiled into the library
 // for grids of up to kNoAllocSms CTAs, so that the call needs no buffer from its caller.
 
