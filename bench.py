@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--workload", choices=("sweep", "attn_pairs", "wide_rows", "prologue_layers"),
                     default="sweep")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--repeats", type=int, default=5,
+                    help="repeats of the K-step timed region; the median is reported")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=0,
@@ -62,17 +64,6 @@ def parse():
     return ap.parse_args()
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) that one ncu capture measured per
-# launch, for layer 0 of the sweep at M = 1 and M = 8 (profiles/nvfp4_gemv_sweep_dram_traffic.md).
-# They describe the kernel code with this SHA-256 only (kernel_code_sha256: comments and blank
-# lines do not count); for any other code the bench reports traffic as null.
-TRAFFIC_SOURCE_SHA256 = "d1b5f55b5d018df462518828592786b8db2e8e99ec64e00852a2de8f26c49be8"
-TRAFFIC_BYTES = {
-    ("L0.qkv", 1): 30119168, ("L0.o", 1): 18324480, ("L0.gate_up", 1): 106684416,
-    ("L0.down", 1): 50807296,
-    ("L0.qkv", 8): 29617152, ("L0.o", 8): 17837312, ("L0.gate_up", 8): 105905152,
-    ("L0.down", 8): 50465024,
-}
 KERNEL_SOURCE = os.path.join(ROOT, "nvfp4_weight_only_03_b200", "csrc", "nvfp4_gemv.cu")
 
 
@@ -87,22 +78,25 @@ def kernel_code_sha256(path: str = KERNEL_SOURCE) -> str:
     return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()
 
 
-def measured_traffic(kind: str, bytes_of: dict, kind_of: dict):
-    """Mean ncu DRAM bytes per launch of `kind` over the captured launches, with the mean
-    algorithmic bytes of the same launches; None when the kernel source has changed since."""
+# DRAM bytes per launch of the chain kernel from one ncu capture (profiles/
+# nvfp4_gemv_chain_dram_traffic.md): layer 0's four projections as one chain at M = 1 and 8,
+# scaled to a full M pass by the weight bytes.  Valid only for the kernel code with this SHA-256.
+CHAIN_TRAFFIC_SHA256 = None
+CHAIN_TRAFFIC_RATIO = None  # measured DRAM bytes / algorithmic bytes of the captured launches
+
+
+def measured_chain_traffic():
     try:
-        if kernel_code_sha256() != TRAFFIC_SOURCE_SHA256:
+        if CHAIN_TRAFFIC_SHA256 is None or kernel_code_sha256() != CHAIN_TRAFFIC_SHA256:
             return None
     except OSError:
         return None
-    keys = [k for k in TRAFFIC_BYTES if kind_of.get(k) == kind]
-    if not keys:
-        return None
-    meas = sum(TRAFFIC_BYTES[k] for k in keys) / len(keys)
-    alg = sum(bytes_of[k] for k in keys) / len(keys)
-    return {"bytes_per_launch": round(meas), "algorithmic_bytes_per_launch": round(alg),
-            "ratio": round(meas / alg, 4),
-            "launches": [f"{n}@M{m}" for (n, m) in keys]}
+    wl = synth.describe(WORKLOAD)
+    bytes_avg = sum(step_bytes(wl).values()) / len(wl.rows)
+    return {"bytes_per_launch": round(bytes_avg * CHAIN_TRAFFIC_RATIO),
+            "ratio": CHAIN_TRAFFIC_RATIO,
+            "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of layer 0 as one chain at "
+                   "M = 1 and 8, as a ratio to its algorithmic bytes, times a full M pass"}
 
 
 def step_bytes(wl) -> dict:
@@ -254,6 +248,21 @@ def cpu_oracle_sample(wl, seconds: float):
 # our arm
 
 
+def sweep_chain_ops(nv, wl, dw, m, x_key="x", y_key="y", x_of=None, y_of=None):
+    """The sweep's 16 projections at M rows as one chain, in sweep order, each with its own x
+    (x_of / y_of map an entry to its x / y tensors when given)."""
+    ops = []
+    for e in dw:
+        p = e["p"]
+        x = x_of(e, m) if x_of else e[x_key][:m]
+        y = y_of(e, m) if y_of else e[y_key][:m]
+        if p.dual:
+            ops.append(nv.ChainOp.dual(e["W"], e["S"], e["g"], e["Wu"], e["Su"], e["gu"], x=x, y=y))
+        else:
+            ops.append(nv.ChainOp.single([(e["W"], e["S"], e["g"])], x=x, ys=[y]))
+    return ops
+
+
 def run_ours(args, world, rank, local):
     import torch
     import nvfp4_weight_only_03_b200 as nv
@@ -262,6 +271,7 @@ def run_ours(args, world, rank, local):
     wl = synth.make(WORKLOAD)
     bytes_of = step_bytes(wl)
     total_step_bytes = sum(bytes_of.values())
+    pass_bytes = {m: sum(bytes_of[(p.name, m)] for p in wl.projections) for m in wl.rows}
 
     # resident inputs
     dw = []
@@ -277,178 +287,175 @@ def run_ours(args, world, rank, local):
         dw.append(ent)
     ws = nv.workspace(dev)
     wsp, wsn = ws.data_ptr(), ws.numel()
-
     flags = nv.FLAG_PREFETCH_WEIGHTS  # decode step: weights are constants
 
-    def launches(stream_handle, x_key="x", y_key="y"):
-        """[(kind, key, fn)] for one step, raw C ABI calls with precomputed arguments."""
+    # the step: one chained launch per M (the 16 projections back to back in one persistent
+    # kernel); every projection's result is bitwise that of its own launch
+    structs = {m: nv._chain_structs(sweep_chain_ops(nv, wl, dw, m)) for m in wl.rows}
+    cbytes = 0
+    for m, (arr, mm, _, _) in structs.items():
+        b = ctypes.c_size_t()
+        st = L.nvfp4_chain_workspace_bytes(arr, len(dw), mm, ctypes.byref(b))
+        if st != 0:
+            raise RuntimeError(f"chain workspace: {nv.STATUS.get(st, st)}")
+        cbytes = max(cbytes, int(b.value))
+    cws = torch.zeros(cbytes, dtype=torch.uint8, device=dev)
+
+    def chain_launches(sh):
+        return [(f"chain@M{m}", m, L.nvfp4_gemv_chain,
+                 (structs[m][0], len(dw), m, cws.data_ptr(), cws.numel(), flags, sh))
+                for m in wl.rows]
+
+    def separate_launches(sh):
+        """The same step as 64 launches (one per projection and M), for comparison."""
         seq = []
         for m in wl.rows:
             for e in dw:
                 p = e["p"]
-                xp, yp = e[x_key].data_ptr(), e[y_key].data_ptr()
+                xp, yp = e["x"].data_ptr(), e["y"].data_ptr()
                 if p.dual:
                     a = (e["W"].data_ptr(), e["S"].data_ptr(), ctypes.c_float(e["g"]),
                          e["Wu"].data_ptr(), e["Su"].data_ptr(), ctypes.c_float(e["gu"]), xp,
-                         p.k, yp, p.n, m, p.n, p.k, wsp, wsn, flags, stream_handle)
+                         p.k, yp, p.n, m, p.n, p.k, wsp, wsn, flags, sh)
                     seq.append(("nvfp4_gemv_dual", (p.name, m), L.nvfp4_gemv_dual_ex, a))
                 else:
                     a = (e["W"].data_ptr(), e["S"].data_ptr(), ctypes.c_float(e["g"]), xp, p.k,
-                         yp, p.n, m, p.n, p.k, wsp, wsn, flags, stream_handle)
+                         yp, p.n, m, p.n, p.k, wsp, wsn, flags, sh)
                     seq.append(("nvfp4_gemv", (p.name, m), L.nvfp4_gemv_ex, a))
         return seq
 
     stream = torch.cuda.Stream(device=dev)
     sh = stream.cuda_stream
-    seq = launches(sh)
 
-    def eager_step():
-        for _, _, fn, a in seq:
-            st = fn(*a)
+    def run_seq(seq):
+        for item in seq:
+            st = item[2](*item[3])
             if st != 0:
                 raise RuntimeError(f"launch failed: {nv.STATUS.get(st, st)}")
 
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
-            eager_step()
+            run_seq(chain_launches(sh))
+            run_seq(separate_launches(sh))
     stream.synchronize()
 
     if args.profile_steps:
         with torch.cuda.stream(stream):
             for _ in range(args.profile_steps):
-                eager_step()
+                run_seq(chain_launches(sh))
         stream.synchronize()
         return None
 
-    # the step as a CUDA graph (the timed region replays it), and a second capture with an
-    # event pair around every launch for the per-kernel durations (the event nodes break the
-    # launches' overlap, so those durations are for launches that run alone)
-    def capture(with_events):
-        ev = None
-        if with_events:
-            try:
-                ev = [(torch.cuda.Event(enable_timing=True, external=True),
-                       torch.cuda.Event(enable_timing=True, external=True)) for _ in seq]
-            except TypeError:
-                return None, None
+    def capture(make, with_events):
+        """A CUDA graph of one step (optionally with an event pair around every launch: those
+        events break the launches' overlap, so their durations are for launches run alone)."""
         graph = torch.cuda.CUDAGraph()
+        ev = None
         with torch.cuda.graph(graph, stream=stream):
             cs = torch.cuda.current_stream().cuda_stream
-            cap = launches(cs)
-            for i, (_, _, fn, a) in enumerate(cap):
+            seq = make(cs)
+            if with_events:
+                ev = [(torch.cuda.Event(enable_timing=True, external=True),
+                       torch.cuda.Event(enable_timing=True, external=True)) for _ in seq]
+            for i, item in enumerate(seq):
                 if ev is not None:
                     ev[i][0].record()
-                st = fn(*a)
+                st = item[2](*item[3])
                 if ev is not None:
                     ev[i][1].record()
                 if st != 0:
                     raise RuntimeError(f"capture failed: {nv.STATUS.get(st, st)}")
-        return graph, ev
+        return graph, ev, seq
 
-    graph, _ = capture(False)
-    graph_ev, ev = capture(True)
-    for _ in range(3):
-        graph.replay()
-        if graph_ev is not None:
-            graph_ev.replay()
+    graph, _, cseq = capture(chain_launches, False)
+    graph_ev, ev, _ = capture(chain_launches, True)
+    graph_sep, _, sseq = capture(separate_launches, False)
+    graph_sep_ev, sev, _ = capture(separate_launches, True)
+    for g in (graph, graph_ev, graph_sep, graph_sep_ev):
+        for _ in range(3):
+            g.replay()
     torch.cuda.synchronize()
+
+    def timed(g, steps):
+        t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            t_begin.record()
+            for _ in range(steps):
+                g.replay()
+            t_end.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(t_begin.elapsed_time(t_end), world)
 
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        t_begin.record()
-        for _ in range(args.steps):
-            graph.replay()
-        t_end.record()
-    torch.cuda.synchronize()
-    barrier(world)
-    ms = t_begin.elapsed_time(t_end)
-    ms = max_over_ranks(ms, world)
-    # per-launch durations: the instrumented step, replayed right after the timed region
-    per_launch = {}
+    # the timed region: K steps, repeated `repeats` times; the median repeat is the number
+    repeats = max(1, args.repeats)
+    rep_ms = [timed(graph, args.steps) for _ in range(repeats)]
+    ms = sorted(rep_ms)[len(rep_ms) // 2]
+    sep_steps = max(1, min(args.steps, 50))
+    sep_ms = timed(graph_sep, sep_steps) / sep_steps
+    # per-launch durations of launches run alone: the instrumented graphs, median of 10 replays
     reps = 10
-    if ev is not None:
-        timing_src = f"events around each launch of a captured step, median of {reps} replays"
-        samples = {key: [] for (_, key, _, _) in seq}
+
+    def launch_us(g, events, seq):
+        samples = [[] for _ in seq]
         for _ in range(reps):
             with torch.cuda.stream(stream):
-                graph_ev.replay()
+                g.replay()
             torch.cuda.synchronize()
-            for (e0, e1), (kind, key, _, _) in zip(ev, seq):
-                samples[key].append(e0.elapsed_time(e1) * 1e3)
-        for kind, key, _, _ in seq:
-            v = sorted(samples[key])
-            per_launch[key] = (kind, v[len(v) // 2])
-    else:
-        timing_src = "events around eager launches"
-        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for _ in seq]
-        with torch.cuda.stream(stream):
-            for (e0, e1), (_, _, fn, a) in zip(pairs, seq):
-                e0.record()
-                fn(*a)
-                e1.record()
-        torch.cuda.synchronize()
-        for (e0, e1), (kind, key, _, _) in zip(pairs, seq):
-            per_launch[key] = (kind, e0.elapsed_time(e1) * 1e3)
+            for i, (e0, e1) in enumerate(events):
+                samples[i].append(e0.elapsed_time(e1) * 1e3)
+        return [sorted(v)[len(v) // 2] for v in samples]
+
+    chain_us = launch_us(graph_ev, ev, cseq)
+    sep_us = launch_us(graph_sep_ev, sev, sseq)
     clk = clocks.stop()
     ms_per_step = ms / args.steps
     value = world * total_step_bytes * args.steps / (ms * 1e-3) / 1e9
 
-    # per-kernel shares and the dominant kernel's roofline
-    by_kind = {}
-    for key, (kind, us) in per_launch.items():
-        d = by_kind.setdefault(kind, {"us": 0.0, "bytes": 0, "launches": 0})
-        d["us"] += us
-        d["bytes"] += bytes_of[key]
-        d["launches"] += 1
-    dom = max(by_kind, key=lambda k: by_kind[k]["us"])
-    d = by_kind[dom]
-    # The step's launches overlap (programmatic dependent launch), so a launch's duration inside
-    # the timed region is the step time apportioned by the kernels' shares of launch time; the
-    # shares come from events around every launch of a second captured copy of the step, whose
-    # launches therefore run one at a time ("isolated").
-    total_us = sum(x["us"] for x in by_kind.values())
-    share = {k: v["us"] / total_us for k, v in by_kind.items()}
-    chain_us = ms_per_step * 1e3 * share[dom] / d["launches"]
-    bytes_avg = d["bytes"] / d["launches"]
-    achieved = bytes_avg / (chain_us * 1e-6) / 1e9
-    iso_us = d["us"] / d["launches"]
-    iso = bytes_avg / (iso_us * 1e-6) / 1e9
+    # the step is 4 launches of one kernel (the chain), back to back: its mean launch duration
+    # inside the timed region is the step time over 4
     peak, peak_src = peaks()
-    kind_of = {key: kind for key, (kind, _) in per_launch.items()}
-    tr = measured_traffic(dom, bytes_of, kind_of)
-    traffic = tr["bytes_per_launch"] if tr else None
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
-                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                "peak_source": peak_src,
-                "traffic_detail": tr,
-                "bytes_per_launch_avg": bytes_avg,
-                "avg_launch_us": round(chain_us, 3),
-                "timing": "CUDA events around the K timed steps on the launching stream; the "
-                          "kernel's launches take its share of the step time",
+    in_step_us = ms_per_step * 1e3 / len(wl.rows)
+    bytes_avg = total_step_bytes / len(wl.rows)
+    achieved = bytes_avg / (in_step_us * 1e-6) / 1e9
+    iso_us = sum(chain_us) / len(chain_us)
+    iso = bytes_avg / (iso_us * 1e-6) / 1e9
+    tr = measured_chain_traffic()
+    roofline = {"bound": "hbm", "kernel": "nvfp4_gemv_chain (nvfp4_gemv_kernel<3>)",
+                "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "traffic": tr["bytes_per_launch"] if tr else None,
+                "peak_source": peak_src, "traffic_detail": tr,
+                "bytes_per_launch_avg": round(bytes_avg), "avg_launch_us": round(in_step_us, 3),
+                "timing": "CUDA events around the K timed steps on the launching stream (median "
+                          f"of {repeats} repeats); a step is 4 chain launches of this kernel",
                 "isolated": {"achieved": round(iso, 1), "frac": round(iso / peak, 4),
-                             "avg_launch_us": round(iso_us, 3), "timing": timing_src},
-                "launch_us_sum_vs_step_us": round(total_us / (ms_per_step * 1e3), 3),
-                "share_of_step": {k: round(v, 4) for k, v in share.items()}}
+                             "avg_launch_us": round(iso_us, 3),
+                             "timing": f"events around each chain launch, median of {reps} "
+                                       "replays"}}
+    per_pass = {}
+    for (name, m, _, _), us in zip(cseq, chain_us):
+        gbps = pass_bytes[m] / (us * 1e-6) / 1e9
+        per_pass[name] = {"us": round(us, 2), "GBps": round(gbps, 1), "frac": round(gbps / peak, 4)}
     detail = {}
-    for (name, m), (kind, us) in sorted(per_launch.items(), key=lambda t: (t[0][1], t[0][0])):
+    for (kind, (name, m), _, _), us in zip(sseq, sep_us):
         b = bytes_of[(name, m)]
         detail[f"{name}@M{m}"] = {"us": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
                                   "frac": round(b / (us * 1e-6) / 1e9 / peak, 4)}
 
     # end to end through the public API: pinned host x in, y out, every step
-    e2e = run_e2e(args, wl, dw, ws, world)
+    e2e = run_e2e(args, wl, dw, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(wl, args.cpu_seconds)
 
-    del graph, graph_ev
+    del graph, graph_ev, graph_sep, graph_sep_ev
     line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -457,24 +464,32 @@ def run_ours(args, world, rank, local):
             "config": {"workload": WORKLOAD_DESC, "seed": wl.seed, "rows": list(wl.rows),
                        "bytes_per_step": total_step_bytes,
                        "l2": "inputs 0.79 GB per M pass > 126 MB L2; no flush",
-                       "launch": "one CUDA graph per step (64 kernels, programmatic dependent "
-                                 "launch between them), persistent grid = SMs",
+                       "launch": "one CUDA graph per step: one chained launch per M (the 16 "
+                                 "projections in one persistent kernel, grid = SMs), "
+                                 "programmatic dependent launch between the 4 launches",
+                       "repeats": rep_ms and [round(x / args.steps, 5) for x in rep_ms],
                        "parallelism": f"replicas x{world}"},
-            "roofline": roofline, "e2e": e2e, "gpu_launches": len(seq) * args.steps,
-            "clocks": clk, "per_launch": detail}
+            "roofline": roofline, "e2e": e2e, "gpu_launches": len(cseq) * args.steps * repeats,
+            "clocks": clk, "per_pass": per_pass,
+            "separate_launches": {
+                "ms_per_step": round(sep_ms, 5),
+                "GBps": round(world * total_step_bytes / (sep_ms * 1e-3) / 1e9, 1),
+                "what": "the same step as 64 launches (nvfp4_gemv_ex / nvfp4_gemv_dual_ex), one "
+                        "CUDA graph with programmatic dependent launch"},
+            "per_launch": detail}
     if cpu is not None:
         line["cpu_baseline"] = cpu
     return line
 
 
-def run_e2e(args, wl, dw, ws, world):
-    """Same metric through the public Python API (`gemv`, `gemv_dual`), as a serving loop runs
-    it.  Every step copies the step's inputs (each projection's x, 8 rows) from pinned host
-    memory to the device in one copy, runs the 64 calls, and reads every call's y back into
-    pinned host memory in one copy; all of it is inside the timed region.  The copies run on
-    their own streams (one for H2D, one for D2H) with two buffers, so one step's copies overlap
-    the neighbouring steps' kernels; events keep every buffer from being overwritten while a
-    copy or kernel still uses it."""
+def run_e2e(args, wl, dw, world):
+    """Same metric through the public Python API (nvfp4_weight_only_03_b200.Chain, one prepared
+    chain per M and buffer), as a serving loop runs it.  Every step copies the step's inputs
+    (each projection's x, 8 rows) from pinned host memory to the device in one copy, runs the
+    4 chains, and reads every projection's y back into pinned host memory in one copy; all of
+    it is inside the timed region.  The copies run on their own streams (one for H2D, one for
+    D2H) with two buffers, so one step's copies overlap the neighbouring steps' kernels; events
+    keep every buffer from being overwritten while a copy or kernel still uses it."""
     import torch
     import nvfp4_weight_only_03_b200 as nv
     dev = dw[0]["x"].device
@@ -500,16 +515,20 @@ def run_e2e(args, wl, dw, ws, world):
     compute = torch.cuda.Stream(device=dev)
     h2d = torch.cuda.Stream(device=dev)
     d2h = torch.cuda.Stream(device=dev)
-    calls = [[], []]
+    chains = [[], []]
     for buf in range(2):
         for m in wl.rows:
-            for e in dw:
+            def x_of(e, m, buf=buf):
                 p = e["p"]
                 xo = x_off[p.name]
-                x = dx[buf][xo:xo + 8 * p.k].view(8, p.k)[:m]
+                return dx[buf][xo:xo + 8 * p.k].view(8, p.k)[:m]
+
+            def y_of(e, m, buf=buf):
+                p = e["p"]
                 yo = y_off[(p.name, m)]
-                y = dy[buf][yo:yo + m * p.n].view(m, p.n)
-                calls[buf].append((e, x, y))
+                return dy[buf][yo:yo + m * p.n].view(m, p.n)
+            chains[buf].append(nv.Chain(sweep_chain_ops(nv, wl, dw, m, x_of=x_of, y_of=y_of),
+                                        stream=compute, prefetch_weights=True))
     x_ready = [torch.cuda.Event() for _ in range(2)]    # H2D of buffer b done
     x_free = [torch.cuda.Event() for _ in range(2)]     # kernels reading dx[b] done
     y_ready = [torch.cuda.Event() for _ in range(2)]    # kernels writing dy[b] done
@@ -527,13 +546,8 @@ def run_e2e(args, wl, dw, ws, world):
         with torch.cuda.stream(compute):
             compute.wait_event(x_ready[b])
             compute.wait_event(y_free[b])
-            for e, x, y in calls[b]:
-                if e["p"].dual:
-                    nv.gemv_dual(e["W"], e["S"], e["g"], e["Wu"], e["Su"], e["gu"], x, y=y, ws=ws,
-                                 stream=compute, prefetch_weights=True)
-                else:
-                    nv.gemv(e["W"], e["S"], e["g"], x, y=y, ws=ws, stream=compute,
-                            prefetch_weights=True)
+            for ch in chains[b]:
+                ch(stream=compute)
             x_free[b].record(compute)
             y_ready[b].record(compute)
         with torch.cuda.stream(d2h):
@@ -563,9 +577,9 @@ def run_e2e(args, wl, dw, ws, world):
     return {"value": round(world * bytes_step * args.e2e_steps / (ms * 1e-3) / 1e9, 1),
             "unit": "GB/s", "h2d_bytes_per_step": hx.numel() * 2,
             "d2h_bytes_per_step": hy[0].numel() * 2, "steps": args.e2e_steps,
-            "api": "nvfp4_weight_only_03_b200.gemv / gemv_dual, one H2D copy of the step's x "
-                   "and one D2H copy of its y per step, copies on their own streams overlapping "
-                   "the neighbouring steps (two buffers)"}
+            "api": "nvfp4_weight_only_03_b200.Chain (one prepared chain per M), one H2D copy of "
+                   "the step's x and one D2H copy of its y per step, copies on their own streams "
+                   "overlapping the neighbouring steps (two buffers)"}
 
 
 # ----------------------------------------------------------------------------------------------

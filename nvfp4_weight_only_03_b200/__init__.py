@@ -471,7 +471,9 @@ def _chain_structs(ops, m_hint=None):
         raise ValueError(f"1..{CHAIN_MAX_OPS} operations, got {n_ops}")
     m = m_hint
     xs = []
-    for op in ops:
+    for i, op in enumerate(ops):
+        if op.x_from is not None and not 0 <= int(op.x_from) < i:
+            raise ValueError(f"operation {i}: x_from must name an earlier operation")
         if op.x is not None:
             k = _weight_args(*op.weights[0][:2])[1]
             x, mm, ldx = _x_args(op.x, k)
@@ -521,24 +523,42 @@ def chain_workspace_bytes(ops, m: int = None) -> int:
     return int(b.value)
 
 
+class Chain:
+    """A chain marshalled once for repeated launches (a serving loop's fixed plan): the ChainOp
+    list's pointers, shapes and outputs are fixed at construction; every call enqueues the whole
+    chain (nvfp4_gemv_chain) on `stream` and returns the outputs, as gemv_chain does."""
+
+    def __init__(self, ops, ws: torch.Tensor = None, stream=None, prefetch_weights: bool = False):
+        ops = list(ops)
+        self._arr, self.m, results, self._keep = _chain_structs(ops)
+        self._count = len(ops)
+        self._keep_ops = ops
+        b = ctypes.c_size_t()
+        _check(lib().nvfp4_chain_workspace_bytes(self._arr, self._count, self.m, ctypes.byref(b)),
+               "nvfp4_chain_workspace_bytes")
+        self.workspace_bytes = int(b.value)
+        dev = results[0][0].device
+        self.ws = ws if ws is not None else _cached_workspace("chain", self.workspace_bytes, dev,
+                                                              stream)
+        if self.ws.numel() < self.workspace_bytes:
+            raise ValueError(f"workspace of {self.ws.numel()} bytes, need {self.workspace_bytes}")
+        self.flags = FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0
+        self.outputs = [r[0] if len(r) == 1 else r for r in results]
+
+    def __call__(self, stream=None, check: bool = False) -> list:
+        st = lib().nvfp4_gemv_chain(self._arr, self._count, self.m, self.ws.data_ptr(),
+                                    self.ws.numel(), self.flags, _stream(stream))
+        _check(st, "nvfp4_gemv_chain")
+        if check:
+            _check_error(self.ws, stream, "nvfp4_gemv_chain")
+        return self.outputs
+
+
 def gemv_chain(ops, ws: torch.Tensor = None, stream=None, prefetch_weights: bool = False,
                check: bool = False) -> list:
     """Runs the ChainOp list in one persistent launch per 8-row pass (nvfp4_gemv_chain).
     Returns, per operation, its output (a tensor) or, for a single operation with several
     weights, the list of its outputs.  Each is bitwise what gemv_multi / gemv_dual gives for
     the same x.  ws, check: as for gemv (the default workspace is grown to the chain's size)."""
-    ops = list(ops)
-    arr, m, results, _keep = _chain_structs(ops)
-    b = ctypes.c_size_t()
-    _check(lib().nvfp4_chain_workspace_bytes(arr, len(ops), m, ctypes.byref(b)),
-           "nvfp4_chain_workspace_bytes")
-    dev = results[0][0].device
-    if ws is None:
-        ws = _cached_workspace("chain", int(b.value), dev, stream)
-    st = lib().nvfp4_gemv_chain(arr, len(ops), m, ws.data_ptr(), ws.numel(),
-                                FLAG_PREFETCH_WEIGHTS if prefetch_weights else 0,
-                                _stream(stream))
-    _check(st, "nvfp4_gemv_chain")
-    if check:
-        _check_error(ws, stream, "nvfp4_gemv_chain")
-    return [r[0] if len(r) == 1 else r for r in results]
+    return Chain(ops, ws=ws, stream=stream, prefetch_weights=prefetch_weights)(stream, check)
+
