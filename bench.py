@@ -61,6 +61,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run this many eager steps and exit (for ncu launch lists)")
+    ap.add_argument("--profile-separate", action="store_true",
+                    help="sweep: profile the step as 64 separate launches instead of 4 chains")
     return ap.parse_args()
 
 
@@ -78,11 +80,11 @@ def kernel_code_sha256(path: str = KERNEL_SOURCE) -> str:
     return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()
 
 
-# DRAM bytes per launch of the chain kernel from one ncu capture (profiles/
-# nvfp4_gemv_chain_dram_traffic.md): layer 0's four projections as one chain at M = 1 and 8,
-# scaled to a full M pass by the weight bytes.  Valid only for the kernel code with this SHA-256.
-CHAIN_TRAFFIC_SHA256 = None
-CHAIN_TRAFFIC_RATIO = None  # measured DRAM bytes / algorithmic bytes of the captured launches
+# DRAM bytes of the chained launches from one ncu capture of a bench step (profiles/
+# nvfp4_gemv_chain_launch_list.md): the 4 launches' dram__bytes_read.sum + dram__bytes_write.sum
+# over their algorithmic bytes.  Valid only for the kernel code with this SHA-256.
+CHAIN_TRAFFIC_SHA256 = "73c6d7bf9657f95a163934d6aa887da9cc5096081aa77133f0b3d27861f112d1"
+CHAIN_TRAFFIC_RATIO = 3276694016 / 3170058240  # 1.0336
 
 
 def measured_chain_traffic():
@@ -95,8 +97,9 @@ def measured_chain_traffic():
     bytes_avg = sum(step_bytes(wl).values()) / len(wl.rows)
     return {"bytes_per_launch": round(bytes_avg * CHAIN_TRAFFIC_RATIO),
             "ratio": CHAIN_TRAFFIC_RATIO,
-            "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of layer 0 as one chain at "
-                   "M = 1 and 8, as a ratio to its algorithmic bytes, times a full M pass"}
+            "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one step's 4 chained "
+                   "launches over their algorithmic bytes, times the mean algorithmic bytes per "
+                   "launch"}
 
 
 def step_bytes(wl) -> dict:
@@ -214,34 +217,41 @@ def max_over_ranks(v: float, world: int) -> float:
 # CPU oracle baseline (bounded sample)
 
 
+SAMPLE_ROWS = 256
+
+
+def oracle_slice(oracle, p, m, rng, threads) -> int:
+    """The fp64 oracle on SAMPLE_ROWS consecutive output rows of projection p at M = m, at a
+    random offset; returns the algorithmic bytes of that slice."""
+    rows = np.arange(0, min(p.n, SAMPLE_ROWS)) + int(rng.integers(0, max(1, p.n - SAMPLE_ROWS)))
+    if p.dual:
+        oracle.gemv_dual(p.w.packed, p.w.scales, p.w.g, p.w_up.packed, p.w_up.scales,
+                         p.w_up.g, p.x[:m], rows=rows, threads=threads)
+    else:
+        oracle.gemv(p.w.packed, p.w.scales, p.w.g, p.x[:m], rows=rows, threads=threads)
+    nw = 2 if p.dual else 1
+    return nw * rows.size * (p.k // 2 + p.k // 16) + m * p.k * 2 + m * rows.size * 2
+
+
 def cpu_oracle_sample(wl, seconds: float):
     """Time the fp64 oracle on row slices of the workload's projections (rank 0, host cores)."""
     import oracle
     oracle.build()
     threads = os.cpu_count() or 1
-    done_bytes, t_total, calls = 0, 0.0, []
+    done_bytes, t_total, n = 0, 0.0, 0
     rng = np.random.default_rng(0)
     order = [(p, m) for m in wl.rows for p in wl.projections]
-    i = 0
-    while t_total < seconds and i < 100000:
-        p, m = order[i % len(order)]
-        i += 1
-        rows = np.arange(0, min(p.n, 256)) + int(rng.integers(0, max(1, p.n - 256)))
+    while t_total < seconds and n < 100000:
+        p, m = order[n % len(order)]
+        n += 1
         t0 = time.perf_counter()
-        if p.dual:
-            oracle.gemv_dual(p.w.packed, p.w.scales, p.w.g, p.w_up.packed, p.w_up.scales,
-                             p.w_up.g, p.x[:m], rows=rows, threads=threads)
-        else:
-            oracle.gemv(p.w.packed, p.w.scales, p.w.g, p.x[:m], rows=rows, threads=threads)
-        dt = time.perf_counter() - t0
-        t_total += dt
-        nw = 2 if p.dual else 1
-        done_bytes += nw * rows.size * (p.k // 2 + p.k // 16) + m * p.k * 2 + m * rows.size * 2
-        calls.append(f"{p.name}@M{m}")
+        done_bytes += oracle_slice(oracle, p, m, rng, threads)
+        t_total += time.perf_counter() - t0
     return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": threads,
             "kind": "oracle",
-            "sample": f"{len(calls)} calls of 256 consecutive output rows each, cycling over the "
-                      f"sweep's projections and M in {{1,2,4,8}} ({t_total:.1f} s)"}
+            "sample": f"{n} calls of {SAMPLE_ROWS} consecutive output rows each at random "
+                      f"offsets, cycling over the sweep's projections and M in {{1,2,4,8}} "
+                      f"({t_total:.1f} s)"}
 
 
 # ----------------------------------------------------------------------------------------------
@@ -333,18 +343,21 @@ def run_ours(args, world, rank, local):
             if st != 0:
                 raise RuntimeError(f"launch failed: {nv.STATUS.get(st, st)}")
 
+    if args.profile_steps:
+        # eager steps only, for ncu: 4 chain launches a step (64 separate launches with
+        # --profile-separate); the first max(W, 3) steps are the warm-up
+        make = separate_launches if args.profile_separate else chain_launches
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 3) + args.profile_steps):
+                run_seq(make(sh))
+        stream.synchronize()
+        return None
+
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
             run_seq(chain_launches(sh))
             run_seq(separate_launches(sh))
     stream.synchronize()
-
-    if args.profile_steps:
-        with torch.cuda.stream(stream):
-            for _ in range(args.profile_steps):
-                run_seq(chain_launches(sh))
-        stream.synchronize()
-        return None
 
     def capture(make, with_events):
         """A CUDA graph of one step (optionally with an event pair around every launch: those
@@ -586,26 +599,26 @@ def run_e2e(args, wl, dw, world):
 # reference arm: the CPU oracle on a bounded sample of the same workload
 
 
+REF_SLICES_PER_STEP = 32  # 2 random 256-row slices of each of the 16 projections per step
+
+
 def run_reference(args, world, rank):
+    """The oracle as it stands on the host cores, on a bounded sample of the sweep: each step is
+    REF_SLICES_PER_STEP slices of 256 consecutive output rows at random offsets (the sampler of
+    cpu_baseline), two per projection, at one M (cycling over 1, 2, 4, 8)."""
     if rank != 0:
         return None
     wl = synth.make(WORKLOAD)
     import oracle
     oracle.build()
-    # each step: the oracle on a bounded slice (256 rows) of one projection, cycling
-    order = [(p, m) for m in wl.rows for p in wl.projections]
     threads = os.cpu_count() or 1
+    rng = np.random.default_rng(0)
+    projs = list(wl.projections)
 
     def step(i):
-        p, m = order[i % len(order)]
-        rows = np.arange(256)
-        if p.dual:
-            oracle.gemv_dual(p.w.packed, p.w.scales, p.w.g, p.w_up.packed, p.w_up.scales,
-                             p.w_up.g, p.x[:m], rows=rows, threads=threads)
-        else:
-            oracle.gemv(p.w.packed, p.w.scales, p.w.g, p.x[:m], rows=rows, threads=threads)
-        nw = 2 if p.dual else 1
-        return nw * 256 * (p.k // 2 + p.k // 16) + m * p.k * 2 + m * 256 * 2
+        m = wl.rows[i % len(wl.rows)]
+        return sum(oracle_slice(oracle, projs[j % len(projs)], m, rng, threads)
+                   for j in range(REF_SLICES_PER_STEP))
 
     for i in range(args.warmup):
         step(i)
@@ -614,15 +627,17 @@ def run_reference(args, world, rank):
     b = sum(step(i) for i in range(steps))
     dt = time.perf_counter() - t0
     v = b / dt / 1e9
+    sample = (f"each step = {REF_SLICES_PER_STEP} slices of {SAMPLE_ROWS} consecutive output rows "
+              f"at random offsets, two per projection, at one M cycling over {{1,2,4,8}} ({steps} "
+              f"steps, {dt:.1f} s); the cpu_baseline sampler")
     return {"metric": METRIC, "value": round(v, 3), "unit": "GB/s", "n_gpus": world,
             "steps": steps, "warmup": args.warmup, "ms_per_step": round(dt / steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD_DESC, "seed": wl.seed, "rows": list(wl.rows)},
+            "config": {"workload": WORKLOAD_DESC, "seed": wl.seed, "rows": list(wl.rows),
+                       "sample": f"{SAMPLE_ROWS}-row slices (a bounded sample of the workload)"},
             "cpu_baseline": {"value": round(v, 3), "unit": "GB/s", "cores": threads,
-                             "kind": "oracle",
-                             "sample": f"each step = 256 output rows of one projection at one M, "
-                                       f"cycling over the sweep ({steps} steps, {dt:.1f} s)"},
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": round(v, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
