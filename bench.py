@@ -461,6 +461,8 @@ def run_ours(args, world, rank, local):
         detail[f"{name}@M{m}"] = {"us": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
                                   "frac": round(b / (us * 1e-6) / 1e9 / peak, 4)}
 
+    mlp = mlp_pairs(nv, L, wl, dw, dev, stream, flags, peak)
+
     # end to end through the public API: pinned host x in, y out, every step
     e2e = run_e2e(args, wl, dw, world)
 
@@ -489,10 +491,71 @@ def run_ours(args, world, rank, local):
                 "GBps": round(world * total_step_bytes / (sep_ms * 1e-3) / 1e9, 1),
                 "what": "the same step as 64 launches (nvfp4_gemv_ex / nvfp4_gemv_dual_ex), one "
                         "CUDA graph with programmatic dependent launch"},
-            "per_launch": detail}
+            "per_launch": detail, "mlp_pair": mlp}
     if cpu is not None:
         line["cpu_baseline"] = cpu
     return line
+
+
+def mlp_pairs(nv, L, wl, dw, dev, stream, flags, peak, replays: int = 50):
+    """The MLP pair of each layer as one chained launch, gate_up dual -> down with down's x the
+    dual's output (x_from, a device-side dependency), at M = 1 and 8: 4 launches (one per
+    layer) in one CUDA graph, median of 5 timings of `replays` replays."""
+    import torch
+    out = {}
+    layers = [(dw[i], dw[i + 1]) for i in range(len(dw) - 1) if dw[i]["p"].dual]
+    for m in (1, 8):
+        acts = [torch.empty((m, gu["p"].n), dtype=torch.bfloat16, device=dev) for gu, _ in layers]
+        structs, wsb = [], 0
+        for (gu, dn), act in zip(layers, acts):
+            ops = [nv.ChainOp.dual(gu["W"], gu["S"], gu["g"], gu["Wu"], gu["Su"], gu["gu"],
+                                   x=gu["x"][:m], y=act),
+                   nv.ChainOp.single([(dn["W"], dn["S"], dn["g"])], x_from=0, ys=[dn["y"][:m]])]
+            st = nv._chain_structs(ops)
+            b = ctypes.c_size_t()
+            if L.nvfp4_chain_workspace_bytes(st[0], 2, st[1], ctypes.byref(b)) != 0:
+                raise RuntimeError("mlp chain workspace")
+            wsb = max(wsb, int(b.value))
+            structs.append((st, ops))
+        ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+
+        def launch(sh):
+            for (arr, mm, _, _), _ in structs:
+                st = L.nvfp4_gemv_chain(arr, 2, mm, ws.data_ptr(), ws.numel(), flags, sh)
+                if st != 0:
+                    raise RuntimeError(f"mlp chain: {nv.STATUS.get(st, st)}")
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                launch(stream.cuda_stream)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            launch(torch.cuda.current_stream().cuda_stream)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record()
+                for _ in range(replays):
+                    g.replay()
+                e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) / replays / len(layers) * 1e3)
+        us = sorted(times)[len(times) // 2]
+        gu, dn = layers[0][0]["p"], layers[0][1]["p"]
+        nbytes = (2 * (gu.n * gu.k // 2 + gu.n * gu.k // 16) + m * gu.k * 2 + m * gu.n * 2 +
+                  dn.n * dn.k // 2 + dn.n * dn.k // 16 + m * dn.k * 2 + m * dn.n * 2)
+        gbps = nbytes / (us * 1e-6) / 1e9
+        out[f"M{m}"] = {"us_per_launch": round(us, 2), "GBps": round(gbps, 1),
+                        "frac": round(gbps / peak, 4), "bytes_per_launch": nbytes}
+        del g
+    out["what"] = ("one nvfp4_gemv_chain launch per layer: gate_up dual 2x17408x5120 -> down "
+                   "5120x17408 reading the dual's output through x_from (cooperative launch); "
+                   "4 layers per CUDA graph, median of 5 x 50 replays")
+    return out
 
 
 def run_e2e(args, wl, dw, world):

@@ -308,3 +308,90 @@ def test_gated_rmsnorm_valid_call_reaches_the_device(L):
     if not cuda_ok():
         assert L.nvfp4_gemv_pro(ctypes.byref(p), PW, PW, 1.0, PX, 256, PY, 64, 2, 64, 256, PWS,
                                 1 << 30, 0, None) == expect
+
+
+# ---- nvfp4_gemv_chain / nvfp4_chain_workspace_bytes: host checks (no CUDA call is reached)
+
+def chain_op(kind=0, outputs=1, n=256, k=256, x=A16, ldx=None, x_from=-1, y=A16, ldy=None,
+             w=A16, s=A16, up=None):
+    op = nv.ChainOpStruct()
+    op.kind, op.outputs, op.k, op.x_from = kind, outputs, k, x_from
+    op.x, op.ldx = x, (k if ldx is None else ldx)
+    for o in range(min(outputs, nv.MAX_OUTPUTS) if kind == 0 else 2):
+        op.out[o].w, op.out[o].s, op.out[o].global_scale = w, s, 1.0
+        op.out[o].y, op.out[o].ldy, op.out[o].n = y, (n if ldy is None else ldy), n
+    if kind == 1 and up is not None:
+        op.out[1].n = up
+    return op
+
+
+def run_chain(L, ops, m=1, ws=A16, wsb=1 << 30, flags=0):
+    arr = (nv.ChainOpStruct * max(1, len(ops)))(*ops)
+    return L.nvfp4_gemv_chain(arr, len(ops), m, ws, wsb, flags, None)
+
+
+@pytest.mark.parametrize("ops,kw,status", [
+    ([chain_op()], dict(m=0), -3),
+    ([chain_op()], dict(m=129), -3),
+    ([chain_op()] * 17, {}, -2),                                   # more than 16 operations
+    ([chain_op(kind=2)], {}, -2),                                  # unknown kind
+    ([chain_op(outputs=0)], {}, -2),
+    ([chain_op(outputs=5)], {}, -2),
+    ([chain_op(k=128)], {}, -2),                                   # K % 256 != 0
+    ([chain_op(x_from=0)], {}, -2),                                # reads itself
+    ([chain_op(), chain_op(x_from=2)], {}, -2),                    # reads a later operation
+    ([chain_op(n=512), chain_op(k=256, x_from=0)], {}, -2),        # source N != this K
+    ([chain_op(outputs=2), chain_op(k=256, x_from=0)], {}, -2),    # source has two outputs
+    ([chain_op(y=A16 + 2), chain_op(x_from=0)], {}, -4),           # source y not 16-byte aligned
+    ([chain_op(ldy=260), chain_op(x_from=0)], {}, -4),             # source ldy % 8 != 0
+    ([chain_op(x=None)], {}, -1),
+    ([chain_op(ldx=128)], {}, -2),
+    ([chain_op(x=A16 + 8)], {}, -4),
+    ([chain_op(w=None)], {}, -1),
+    ([chain_op(y=None)], {}, -1),
+    ([chain_op(s=A16 + 2)], {}, -4),                               # scales move by TMA
+    ([chain_op(kind=1, up=128)], {}, -2),                          # dual: up N != gate N
+    ([chain_op()], dict(flags=4), -2),                             # unknown flag
+    ([chain_op()], dict(ws=None), -7),
+    ([chain_op()], dict(ws=A16 + 4), -7),
+])
+def test_chain_host_argument_checks(L, ops, kw, status):
+    assert run_chain(L, ops, **kw) == status
+
+
+def test_chain_null_ops_and_workspace_query_checks(L):
+    assert L.nvfp4_gemv_chain(None, 1, 1, A16, 1 << 30, 0, None) == -1
+    b = ctypes.c_size_t()
+    assert L.nvfp4_chain_workspace_bytes(None, 1, 1, ctypes.byref(b)) == -1
+    arr = (nv.ChainOpStruct * 1)(chain_op())
+    assert L.nvfp4_chain_workspace_bytes(arr, 1, 1, None) == -1
+    assert L.nvfp4_chain_workspace_bytes(arr, 0, 1, ctypes.byref(b)) == -2
+    assert L.nvfp4_chain_workspace_bytes(arr, 1, 200, ctypes.byref(b)) == -3
+    # the test hook checks its limit before anything else
+    assert L.nvfp4_gemv_chain_unsignalled(arr, 1, 1, A16, 1 << 30, 0, None) == -2
+    assert L.nvfp4_gemv_chain_unsignalled(arr, 1, 1, A16, 1 << 30, 2 * 10 ** 9, None) == -2
+
+
+@pytest.mark.skipif(cuda_ok(), reason="only meaningful on a host without a CUDA device")
+def test_valid_chain_without_device_reports_arch(L):
+    assert run_chain(L, [chain_op(), chain_op(n=256, x_from=0)]) == -5
+
+
+def test_chain_binding_argument_checks():
+    t = torch_cpu_bf16((1, 256))
+    w = torch_cpu_u8((256, 128))
+    s = torch_cpu_u8((256, 16))
+    with pytest.raises((ValueError, TypeError)):
+        nv.ChainOp.single([(w, s, 1.0)], x=t, x_from=0)          # both x and x_from
+    with pytest.raises((ValueError, TypeError)):
+        nv._chain_structs([nv.ChainOp.single([(w, s, 1.0)], x_from=0)])  # reads itself
+
+
+def torch_cpu_bf16(shape):
+    import torch
+    return torch.zeros(shape, dtype=torch.bfloat16)
+
+
+def torch_cpu_u8(shape):
+    import torch
+    return torch.zeros(shape, dtype=torch.uint8)
