@@ -662,13 +662,13 @@ def run_e2e(args, wl, dw, world):
 # reference arm: the CPU oracle on a bounded sample of the same workload
 
 
-REF_SLICES_PER_STEP = 32  # 2 random 256-row slices of each of the 16 projections per step
+REF_SLICES_PER_STEP = 48  # 3 random 256-row slices of each of the 16 projections per step
 
 
 def run_reference(args, world, rank):
     """The oracle as it stands on the host cores, on a bounded sample of the sweep: each step is
     REF_SLICES_PER_STEP slices of 256 consecutive output rows at random offsets (the sampler of
-    cpu_baseline), two per projection, at one M (cycling over 1, 2, 4, 8)."""
+    cpu_baseline), three per projection, at one M (cycling over 1, 2, 4, 8)."""
     if rank != 0:
         return None
     wl = synth.make(WORKLOAD)
@@ -691,7 +691,7 @@ def run_reference(args, world, rank):
     dt = time.perf_counter() - t0
     v = b / dt / 1e9
     sample = (f"each step = {REF_SLICES_PER_STEP} slices of {SAMPLE_ROWS} consecutive output rows "
-              f"at random offsets, two per projection, at one M cycling over {{1,2,4,8}} ({steps} "
+              f"at random offsets, three per projection, at one M cycling over {{1,2,4,8}} ({steps} "
               f"steps, {dt:.1f} s); the cpu_baseline sampler")
     return {"metric": METRIC, "value": round(v, 3), "unit": "GB/s", "n_gpus": world,
             "steps": steps, "warmup": args.warmup, "ms_per_step": round(dt / steps * 1e3, 3),
