@@ -669,6 +669,9 @@ __device__ __forceinline__ void consume_op(const LP& L, const Op& op, uint8_t* r
 
     // this lane's weight rows inside a tile (fragment rows g and g+8)
     const int pr_a = perm_row(g), pr_b = perm_row(g + 8);
+    // this lane's x row: the mma's column g.  Columns g >= M are computed from row 0 and never
+    // stored (partial tiles and outputs keep columns < M only), so the loads need no predicate.
+    const uint4* const xrow_g = xsm + (g < m ? g : 0) * xrow + q * 4;
     const int frag = (warp * 32 + lane) * 4;  // this lane's floats in a partial tile
 
     float acc[NS][2][4];
@@ -707,9 +710,7 @@ __device__ __forceinline__ void consume_op(const LP& L, const Op& op, uint8_t* r
             // the unit's two 128-k blocks: chunks 4h .. 4h+3 of each 128-byte row
             uint4 xv[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                xv[j] = g < m ? xsm[g * xrow + (2 * uslot + h) * kSlotU4 + q * 4 + (j ^ q)]
-                              : make_uint4(0, 0, 0, 0);
+            for (int j = 0; j < 4; ++j) xv[j] = xrow_g[(2 * uslot + h) * kSlotU4 + (j ^ q)];
             uint4 wa[NS], wb[NS];
             uint32_t sa[NS], sb[NS];
 #pragma unroll
