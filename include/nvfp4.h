@@ -365,6 +365,15 @@ int nvfp4_gemv_chain_unsignalled(const nvfp4_chain_op_t* ops, int count, int m, 
                                  size_t workspace_bytes, int64_t wait_limit_ns,
                                  cudaStream_t stream);
 
+/* Test form of nvfp4_gemv_chain, for the hand-off of cut row groups: the CTA holding a group's
+ * first unit waits at most owner_wait_ns (0 .. 50000) for the later CTAs' partial sums before it
+ * publishes its own and leaves the group to the last of them (50000 is nvfp4_gemv_chain's
+ * limit).  With 0 nearly every cut group takes that path.  Results are bitwise those of
+ * nvfp4_gemv_chain.  No other use. */
+int nvfp4_gemv_chain_owner_wait(const nvfp4_chain_op_t* ops, int count, int m, void* workspace,
+                                size_t workspace_bytes, int64_t owner_wait_ns,
+                                cudaStream_t stream);
+
 /* Workspace bytes of an nvfp4_gemv_ex / _pro, nvfp4_gemv_dual_ex / _pro or nvfp4_gemv_multi /
  * _pro (the largest of its outputs' sizes) call of M rows with
  * NVFP4_FLAG_WIDE_TENSOR or an input prologue: the nvfp4_workspace_bytes layout followed by the

@@ -179,6 +179,7 @@ def lib():
         L.nvfp4_chain_workspace_bytes.argtypes = [cp, c_int, c_int, ctypes.POINTER(sz)]
         L.nvfp4_gemv_chain.argtypes = [cp, c_int, c_int, vp, sz, ctypes.c_uint32, vp]
         L.nvfp4_gemv_chain_unsignalled.argtypes = [cp, c_int, c_int, vp, sz, i64, vp]
+        L.nvfp4_gemv_chain_owner_wait.argtypes = [cp, c_int, c_int, vp, sz, i64, vp]
         L.nvfp4_status_string.argtypes = [c_int]
         L.nvfp4_status_string.restype = ctypes.c_char_p
         for f in (L.nvfp4_pack_info, L.nvfp4_workspace_bytes, L.nvfp4_gemv, L.nvfp4_gemv_dual,
@@ -186,7 +187,7 @@ def lib():
                   L.nvfp4_gemv_multi, L.nvfp4_workspace_error, L.nvfp4_workspace_bytes_wide,
                   L.nvfp4_gemv_pro, L.nvfp4_gemv_dual_pro, L.nvfp4_gemv_multi_pro,
                   L.nvfp4_chain_workspace_bytes, L.nvfp4_gemv_chain,
-                  L.nvfp4_gemv_chain_unsignalled):
+                  L.nvfp4_gemv_chain_unsignalled, L.nvfp4_gemv_chain_owner_wait):
             f.restype = c_int
         _lib = L
     return _lib

@@ -167,6 +167,7 @@ struct Launch {
                                     // producer lanes copy the scale codes themselves
     int signals;                    // some operation signals completion (chains)
     int64_t wait_ns;                // limit of a dependency wait
+    int64_t owner_wait_ns;          // limit of an owner's wait for the later CTAs' tiles
     uint32_t* done;                 // [kMaxChainOps] completion counts
     uint32_t* exit_count;
     int32_t* error;
@@ -782,7 +783,7 @@ __device__ __forceinline__ void consume_op(const LP& L, const Op& op, uint8_t* r
                                 all = true;
                                 break;
                             }
-                            if ((int64_t)(global_ns() - t0) > kOwnerWaitNs) break;
+                            if ((int64_t)(global_ns() - t0) > L.owner_wait_ns) break;
                             __nanosleep(32);
                         }
                         s_last[1] = all;
@@ -1466,6 +1467,7 @@ int launch_spans(const Span* sp, int count, const void* x, int64_t ldx, int m, i
     L.full_count = scale_mode == kScaleTma ? 1 : 1 + 32;
     L.signals = 0;
     L.wait_ns = kDefaultWaitNs;
+    L.owner_wait_ns = kOwnerWaitNs;
     L.done = reinterpret_cast<uint32_t*>(wsb + kDoneOffset);
     L.exit_count = reinterpret_cast<uint32_t*>(wsb + 4);
     L.error = reinterpret_cast<int32_t*>(wsb);
@@ -1671,6 +1673,7 @@ size_t chain_layout(const ChainPiece* pieces, int np, int sms, size_t* off) {
 int launch_chain_pass(const nvfp4_chain_op_t* ops, int count, const ChainPiece* pieces, int np,
                       const int64_t* groups_of, int r0, int m, int sms, void* ws,
                       const size_t* off, uint32_t flags, int64_t wait_ns, int unsignalled,
+                      int64_t owner_wait_ns,
                       cudaStream_t stream) {
     // LaunchOf<kModeChain> is about 13 KB: keep it off the stack of small host threads
     static thread_local LaunchOf<kModeChain> L;
@@ -1723,6 +1726,7 @@ int launch_chain_pass(const nvfp4_chain_op_t* ops, int count, const ChainPiece* 
     L.full_count = 1;
     L.signals = waits ? 1 : 0;
     L.wait_ns = wait_ns;
+    L.owner_wait_ns = owner_wait_ns;
     L.done = reinterpret_cast<uint32_t*>(wsb + kDoneOffset);
     L.exit_count = reinterpret_cast<uint32_t*>(wsb + 4);
     L.error = reinterpret_cast<int32_t*>(wsb);
@@ -1735,7 +1739,8 @@ int launch_chain_pass(const nvfp4_chain_op_t* ops, int count, const ChainPiece* 
 }
 
 int run_chain(const nvfp4_chain_op_t* ops, int count, int m, void* ws, size_t ws_bytes,
-              uint32_t flags, int64_t wait_ns, int unsignalled, cudaStream_t stream) {
+              uint32_t flags, int64_t wait_ns, int unsignalled, int64_t owner_wait_ns,
+              cudaStream_t stream) {
     if (flags & ~(uint32_t)NVFP4_FLAG_PREFETCH_WEIGHTS) return NVFP4_ERR_SHAPE;
     ChainPiece pieces[kMaxChainOps];
     int np = 0;
@@ -1753,7 +1758,7 @@ int run_chain(const nvfp4_chain_op_t* ops, int count, int m, void* ws, size_t ws
     for (int r0 = 0; r0 < m; r0 += NVFP4_PASS_ROWS) {
         const int rows = m - r0 < NVFP4_PASS_ROWS ? m - r0 : NVFP4_PASS_ROWS;
         if ((st = launch_chain_pass(ops, count, pieces, np, groups_of, r0, rows, di->sms, ws, off,
-                                    flags, wait_ns, unsignalled, stream)) != NVFP4_OK)
+                                    flags, wait_ns, unsignalled, owner_wait_ns, stream)) != NVFP4_OK)
             return st;
     }
     return NVFP4_OK;
@@ -2049,14 +2054,24 @@ int nvfp4_chain_workspace_bytes(const nvfp4_chain_op_t* ops, int count, int m, s
 
 int nvfp4_gemv_chain(const nvfp4_chain_op_t* ops, int count, int m, void* workspace,
                      size_t workspace_bytes, uint32_t flags, cudaStream_t stream) {
-    return run_chain(ops, count, m, workspace, workspace_bytes, flags, kDefaultWaitNs, 0, stream);
+    return run_chain(ops, count, m, workspace, workspace_bytes, flags, kDefaultWaitNs, 0,
+                     kOwnerWaitNs, stream);
 }
 
 int nvfp4_gemv_chain_unsignalled(const nvfp4_chain_op_t* ops, int count, int m, void* workspace,
                                  size_t workspace_bytes, int64_t wait_limit_ns,
                                  cudaStream_t stream) {
     if (wait_limit_ns <= 0 || wait_limit_ns > kDefaultWaitNs) return NVFP4_ERR_SHAPE;
-    return run_chain(ops, count, m, workspace, workspace_bytes, 0u, wait_limit_ns, 1, stream);
+    return run_chain(ops, count, m, workspace, workspace_bytes, 0u, wait_limit_ns, 1,
+                     kOwnerWaitNs, stream);
+}
+
+int nvfp4_gemv_chain_owner_wait(const nvfp4_chain_op_t* ops, int count, int m, void* workspace,
+                                size_t workspace_bytes, int64_t owner_wait_ns,
+                                cudaStream_t stream) {
+    if (owner_wait_ns < 0 || owner_wait_ns > kOwnerWaitNs) return NVFP4_ERR_SHAPE;
+    return run_chain(ops, count, m, workspace, workspace_bytes, 0u, kDefaultWaitNs, 0,
+                     owner_wait_ns, stream);
 }
 
 int nvfp4_workspace_bytes_wide(int64_t n, int64_t k, int m, size_t* bytes) {

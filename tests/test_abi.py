@@ -395,3 +395,10 @@ def torch_cpu_bf16(shape):
 def torch_cpu_u8(shape):
     import torch
     return torch.zeros(shape, dtype=torch.uint8)
+
+
+def test_owner_wait_hook_checks_its_limit(L):
+    arr = (nv.ChainOpStruct * 1)(chain_op())
+    assert L.nvfp4_gemv_chain_owner_wait(arr, 1, 1, A16, 1 << 30, -1, None) == -2
+    assert L.nvfp4_gemv_chain_owner_wait(arr, 1, 1, A16, 1 << 30, 50001, None) == -2
+    assert L.nvfp4_gemv_chain_owner_wait(arr, 1, 0, A16, 1 << 30, 0, None) == -3

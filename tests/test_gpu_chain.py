@@ -211,7 +211,7 @@ def test_bounded_wait_gives_up_and_the_device_stays_usable():
     torch.cuda.synchronize()
     assert np.array_equal(bits(o), bits(o_sep)) and np.array_equal(bits(y), bits(y_sep))
     o_ref, yg, yu, ag, au = oracle.gemv_dual(g.packed, g.scales, g.g, u.packed, u.scales, u.g, x)
-    check_dual(bits(o), o_ref, yg, yu, ag, au, "after the timeout")
+    check_dual(bits(o), o_ref, yg, yu, ag, au, "dual, fresh workspace after a timed-out launch")
 
 
 def test_chain_argument_checks():
@@ -268,3 +268,36 @@ def test_concurrent_streams_with_default_workspaces():
     check_single(want[0], ref, a, "inproj, two streams")
     for st in (s1, s2):
         assert nv.workspace_error(nv.workspace(stream=st), st) == 0
+
+
+@pytest.mark.parametrize("m", [1, 8])
+def test_owner_handoff_is_bitwise_the_normal_path(layer0, m):
+    """Owners that do not wait at all (test hook, limit 0) publish their own partial tile and
+    leave nearly every cut row group to the last of its later CTAs, which finishes it.  Results
+    must be bitwise those of the normal chain, for the layer (single and dual operations) and for
+    the MLP pair reading the dual's output, launch after launch on one workspace (a hand-off
+    word left non-zero would break the next launch)."""
+    from gpu_util import assert_ws_clean
+    qkv, o, gu, down = layer0
+    Wd, Sd, gd = dev_weight(down.w)
+    mlp = [nv.ChainOp.dual(*dev_weight(gu.w), *dev_weight(gu.w_up), x=dev_x(gu.x[:m])),
+           nv.ChainOp.single([(Wd, Sd, gd)], x_from=0)]
+    stream = torch.cuda.current_stream().cuda_stream
+    for chain in (layer_ops(layer0, m, "cuda"), mlp):
+        want = chain_bits(chain)
+        arr, mm, results, keep = nv._chain_structs(chain)
+        ws = torch.zeros(nv.chain_workspace_bytes(chain), dtype=torch.uint8, device="cuda")
+        for limit in (0, 0, 0, 50000):
+            for r in results:
+                for t in r:
+                    t.fill_(0)
+            st = nv.lib().nvfp4_gemv_chain_owner_wait(arr, len(chain), mm, ws.data_ptr(),
+                                                       ws.numel(), limit, stream)
+            assert st == 0, nv.STATUS.get(st, st)
+            torch.cuda.synchronize()
+            assert nv.workspace_error(ws) == 0
+            got = [bits(r[0]) if len(r) == 1 else [bits(t) for t in r] for r in results]
+            for i, (a, b) in enumerate(zip(got, want)):
+                assert np.array_equal(np.asarray(a), np.asarray(b)), \
+                    f"operation {i}, owner limit {limit} ns, M={m}: differs from the normal chain"
+            assert_ws_clean(ws)
