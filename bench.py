@@ -83,8 +83,8 @@ def kernel_code_sha256(path: str = KERNEL_SOURCE) -> str:
 # DRAM bytes of the chained launches from one ncu capture of a bench step (profiles/
 # nvfp4_gemv_chain_launch_list.md): the 4 launches' dram__bytes_read.sum + dram__bytes_write.sum
 # over their algorithmic bytes.  Valid only for the kernel code with this SHA-256.
-CHAIN_TRAFFIC_SHA256 = "73c6d7bf9657f95a163934d6aa887da9cc5096081aa77133f0b3d27861f112d1"
-CHAIN_TRAFFIC_RATIO = 3276694016 / 3170058240  # 1.0336
+CHAIN_TRAFFIC_SHA256 = "ba59ccfc8baf16c591ff876a6207e92e4545634b80307fedda4e988085dfa21e"
+CHAIN_TRAFFIC_RATIO = 3281237760 / 3170058240  # 1.0351
 
 
 def measured_chain_traffic():
