@@ -2,28 +2,32 @@
 // the plan's wider multi_seq arms of up to 128 rows ("Blueprint - circuit executor" page for
 // qwen3.8-27b-nvfp4 on GB10, table "Plan arms"; planner setting w4a16_tc=on).  From about 32
 // rows the contraction outgrows the warp-level mma of the 1..8-row kernel, so this tier uses
-// the 5th-generation tensor cores: tcgen05.mma kind::f16 with bf16 operands, accumulators in
-// tensor memory.
+// the 5th-generation tensor cores: tcgen05.mma kind::f16 with f16 operands (A the decoded
+// weights, B the f16 copy of x), fp32 accumulators in tensor memory.
 //
-//   D[n][m] = sum_k W(n, k) * x[m][k]    (128 weight rows n of a tile by 128 x rows m)
+//   D[n][m] = sum_k W(n, k) * x'[m][k]    (128 weight rows n of a tile by N x rows m)
 //
+// * x': nvfp4_tc_prep writes an f16 copy of x to the workspace (after the call's prologue, if
+//   any), row m scaled by the power of two 2^e(m) that puts its largest magnitude in
+//   [2^14, 2^15), and the row's descale 2^-e(m); the epilogues multiply by it.
 // * Work: a tile is 128 weight rows; K is cut into `splits` equal ranges of 256-k units, and
-//   each CTA computes one (tile, split) item.  The split depends only on (N, K, SM count).
-//   With one split the CTA writes y; otherwise it writes fp32 partials to the workspace and
-//   nvfp4_tc_reduce adds the splits in order (the dual: nvfp4_tc_dual_finish, over both
-//   streams).  Deterministic, no atomics.
-// * Per 64-k stage a producer warp loads, with TMA (no multicast): the x tile (128 rows x 64 k
-//   of bf16, 128-byte swizzle: the MMA's K-major B layout; rows >= M read as zero), the 128
-//   weight rows' packed nibbles (32 bytes each) and the 256-k unit's scale codes.
-// * Four decode warps turn the nibbles into bf16 weights: cvt e2m1x2 -> f16x2, times the e4m3
-//   scale in f16 (exact: at most 6 significant bits), widened to bf16x2 through f32 (exact),
-//   stored as the MMA's K-major A tile (128-byte swizzle) in one of two buffers.
-// * One MMA warp issues 4 x tcgen05.mma (M = 128, N = 128, K = 16) per stage into one fp32
-//   accumulator of 128 tensor-memory columns, and frees the stage and the A buffer with
-//   tcgen05.commit.  The decode warps then read the accumulator (tcgen05.ld) and write out.
-// * Every x row is computed by the same instructions whatever M is (N = 128 always; rows >= M
-//   are zero), so rows are bitwise invariant for every M in 9..128.  Against calls of 1..8
-//   rows (a different instruction sequence and operand type) rows agree within the tolerance.
+//   each CTA (two per SM) computes one (tile, split) item.  The split depends only on (N, K,
+//   SM count).  With one split the CTA writes y; otherwise it writes fp32 partials to the
+//   workspace and nvfp4_tc_reduce adds the splits in order (the dual: nvfp4_tc_dual_finish,
+//   over both streams).  Deterministic, no atomics.
+// * A producer warp loads with TMA (no multicast), per 256-k unit the 128 weight rows' packed
+//   nibbles (128 bytes each, 128-byte swizzle) and scale codes, and per 64-k stage the x' tile
+//   (N rows x 64 k of f16, 128-byte swizzle: the MMA's K-major B layout; rows >= M read as zero).
+// * Eight decode warps (two threads per weight row) turn each stage's nibbles into f16 weights:
+//   cvt e2m1x2 -> f16x2 times the e4m3 scale in f16 (exact: at most 6 significant bits), stored
+//   as the MMA's K-major A tile (128-byte swizzle) in one of NVFP4_TC_ABUF buffers.
+// * One MMA thread issues 4 x tcgen05.mma (M = 128, N = M rounded up to 16, K = 16) per stage
+//   into one fp32 accumulator of up to 128 tensor-memory columns, and frees the stage and the A
+//   buffer with tcgen05.commit.  Four warps then read the accumulator (tcgen05.ld) and write out.
+// * Every x row is computed by the same instructions whatever M is (the MMA's columns do not
+//   depend on each other), so rows are bitwise invariant for every M in 9..128.  Against calls of
+//   1..8 rows (a different instruction sequence and a different x scaling) rows agree within the
+//   tolerance.
 // * Waits are bounded: a wait that gives up records an error in the workspace's error word,
 //   and tensor memory is freed on every path.
 #include <cuda.h>
