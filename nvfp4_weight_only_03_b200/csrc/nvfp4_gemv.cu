@@ -146,6 +146,9 @@ struct Op {
     int wait_idx;                   // completion count to wait for before reading x, or -1
     uint32_t wait_target;           // row groups that count must reach
     int sig_idx;                    // completion count this operation adds to, or -1
+    int rot;                        // the launch's CTA c works on range (c + rot) mod grid: a
+                                    // chain turns the ranges by operation, so that no SM keeps
+                                    // the same hand-off role in every layer
     const uint8_t* s[kMaxOutputs];  // scale codes, per output (dual: per stream)
     float g[kMaxOutputs];           // global scales, per output (dual: per stream)
     uint16_t* y[kMaxOutputs];       // outputs (dual: y[0])
@@ -905,10 +908,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int w = lane; w < kOpWords; w += 32) reinterpret_cast<uint32_t*>(&s_op[0])[w] = src[w];
                 __syncwarp();
                 const Op& op = s_op[0];
+                const int lc = cta + op.rot < (int)gridDim.x ? cta + op.rot : cta + op.rot - (int)gridDim.x;
                 if (op.dual)
-                    produce_op<true, false>(L, op, ring, full_bar, empty_bar, &xreq_bar, r, ok, pol, cta, lane);
+                    produce_op<true, false>(L, op, ring, full_bar, empty_bar, &xreq_bar, r, ok, pol, lc, lane);
                 else
-                    produce_op<false, true>(L, op, ring, full_bar, empty_bar, &xreq_bar, r, ok, pol, cta, lane);
+                    produce_op<false, true>(L, op, ring, full_bar, empty_bar, &xreq_bar, r, ok, pol, lc, lane);
                 __syncwarp();  // every lane is done with this copy
             }
         }
@@ -932,10 +936,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int w = tid; w < kOpWords; w += kConsumers) reinterpret_cast<uint32_t*>(&s_op[1])[w] = src[w];
             named_barrier(1, kConsumers);
             const Op& op = s_op[1];
+            const int lc = cta + op.rot < (int)gridDim.x ? cta + op.rot : cta + op.rot - (int)gridDim.x;
             if (op.dual)
-                consume_op<true, false>(L, op, ring, full_bar, empty_bar, &xreq_bar, xreq_sent, xsm, cr, ok, s_amax, s_descale, s_last, cta, tid);
+                consume_op<true, false>(L, op, ring, full_bar, empty_bar, &xreq_bar, xreq_sent, xsm, cr, ok, s_amax, s_descale, s_last, lc, tid);
             else
-                consume_op<false, true>(L, op, ring, full_bar, empty_bar, &xreq_bar, xreq_sent, xsm, cr, ok, s_amax, s_descale, s_last, cta, tid);
+                consume_op<false, true>(L, op, ring, full_bar, empty_bar, &xreq_bar, xreq_sent, xsm, cr, ok, s_amax, s_descale, s_last, lc, tid);
         }
     }
     if (!xreq_sent) pdl_wait();  // a CTA without units in any operation
@@ -1718,6 +1723,7 @@ int launch_chain_pass(const nvfp4_chain_op_t* ops, int count, const ChainPiece* 
             waits = true;
         }
         if (read[c.src] && !(unsignalled && c.src == first_read)) op.sig_idx = c.src;
+        op.rot = (int)(((int64_t)p * 29) % sms);
         const size_t xb = op_x_bytes(op, m);
         if (xb > xmax) xmax = xb;
     }
