@@ -1723,7 +1723,7 @@ int launch_chain_pass(const nvfp4_chain_op_t* ops, int count, const ChainPiece* 
             waits = true;
         }
         if (read[c.src] && !(unsignalled && c.src == first_read)) op.sig_idx = c.src;
-        op.rot = (int)(((int64_t)p * 29) % sms);
+        op.rot = p % sms;
         const size_t xb = op_x_bytes(op, m);
         if (xb > xmax) xmax = xb;
     }
