@@ -291,12 +291,14 @@ def bf16_ulp_distance(a_bits, b_bits) -> np.ndarray:
 
 def silu(t):
     t = np.asarray(t, np.float64)
-    return t / (1.0 + np.exp(-t))
+    with np.errstate(over="ignore"):  # e^-t = inf for t < -709 gives the exact limit, -0
+        return t / (1.0 + np.exp(-t))
 
 
 def silu_grad(t):
     t = np.asarray(t, np.float64)
-    s = 1.0 / (1.0 + np.exp(-t))
+    with np.errstate(over="ignore"):  # e^-t = inf gives s = 0, the exact limit
+        s = 1.0 / (1.0 + np.exp(-t))
     return s * (1.0 + t * (1.0 - s))
 
 
